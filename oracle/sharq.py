@@ -25,9 +25,10 @@ The pages give no equations. Where they are silent the oracle takes these readin
   lower pair index. This is the pattern the sm_100a sparse FP4 MMA accepts.
 * mask ``elem24``: in every group of 4 keep the 2 largest |x|, ties to the lower index.
 * NVFP4 tensor scale s_g = amax|X| / (6*448) in float32; block scale
-  sf = E4M3_rne_satfinite((a / 6) / s_g); d = E4M3(sf) * s_g; code = E2M1_rne(x / d)
-  (code 0 when d == 0). Dequantised value deq = (E2M1(q) * E4M3(sf)) * s_g, all in
-  float32 with one rounding per operation.
+  sf = E4M3_rne_satfinite((a / 6) / s_g); d = E4M3(sf) * s_g; inv = 1 / d (one
+  correctly rounded reciprocal per block); code = E2M1_rne(x * inv) (code 0 when d == 0).
+  Dequantised value deq = (E2M1(q) * E4M3(sf)) * s_g, all in float32 with one rounding
+  per operation.
 * MXFP4 (OCP MX): e = clamp(floor(log2 a) - 2, -127, 127), scale 2^e as E8M0 code
   e+127, code = E2M1_rne(x * 2^-e); a == 0 gives code 0 for scale and elements.
 * Block domains (forced by the MMA that consumes each operand): the residual uses
@@ -110,8 +111,10 @@ def quant_blocks_nv(v: np.ndarray, s_g: np.float32):
     sf = F.e4m3_encode_unsigned(t.astype(F32))
     sf_val = F.e4m3_decode(sf).astype(F32)  # exact
     d = (sf_val * s_g).astype(F32)
+    # one correctly rounded reciprocal per block, then one float32 product per element
     with np.errstate(divide="ignore", invalid="ignore"):
-        ratio = (v / d[..., None]).astype(F32)
+        inv = (F32(1.0) / d).astype(F32)
+        ratio = (v * inv[..., None]).astype(F32)
     codes = np.where(d[..., None] > 0, F.e2m1_encode(np.where(d[..., None] > 0, ratio, 0)), 0)
     codes = codes.astype(np.uint8)
     q_val = F.e2m1_decode(codes).astype(F32)

@@ -148,7 +148,9 @@ def test_nvfp4_scale_and_codes_are_nearest():
     best = np.abs(np.minimum(t, 448)[..., None] - F.E4M3_TABLE).min(-1)
     assert np.array_equal(np.abs(np.minimum(t, 448) - F.e4m3_decode(sf)), best)
     d = (F.e4m3_decode(sf).astype(np.float32) * s_g).astype(np.float32)
-    _nearest_value_check(v, codes, d[..., None].astype(np.float64))
+    inv = (np.float32(1) / d).astype(np.float32)
+    # codes: nearest grid point of the float32 product x * (1/d)
+    _nearest_value_check((v * inv[..., None]).astype(np.float32), codes, 1.0)
     # the block's largest element lands on the top code (6) for normal-range scales
     amax_pos = np.argmax(np.abs(v), -1)
     top = np.take_along_axis(codes, amax_pos[..., None], -1)[..., 0] & 7
