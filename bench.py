@@ -1,0 +1,339 @@
+#!/usr/bin/env python
+"""Benchmark of the SharQ sparse-dense FP4 linear layer on B200.
+
+One step = the whole hot path on one batch: activation preparation (tensor amax pass +
+fused mask / FP4 quantisation / residual / metadata kernel) and the fused sparse + dense
+FP4 GEMM with its bf16 epilogue. The weight is quantised once, before timing (it is an
+offline step). Inputs are seeded synthetic tensors with the workloads' shapes and value
+distributions (workloads/), resident in HBM before the timed region; several input sets
+rotate so that every step reads operands that are not in L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mlp_gate_up]
+    python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Multi-GPU (torchrun): every rank runs its own batch (independent token batches, no
+collective on the data path); value = all ranks' FLOPs / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SharQ linear TFLOPS (2MNK/t) and % FP4 peak; prep kernel HBM GB/s"
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+PREP_BYTES_PER_ELEM = {"pair48": 2 + 0.25 + 0.0625 + 0.0625 + 0.5 + 0.0625,
+                       "elem24": 2 + 0.5 + 0.0625 + 0.125 + 0.5 + 0.0625}
+
+WORKLOADS = {
+    # name: (M, K, N, per_row_outliers)
+    "mlp_gate_up": (4096, 4096, 14336, False),
+    "attn_proj": (2048, 4096, 4096, False),
+    "mlp_down": (4096, 14336, 4096, True),
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def src_hash(files):
+    h = hashlib.sha1()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+GEMM_SRC = ["fp4_sparse_dense_b200/csrc/gemm.cu", "fp4_sparse_dense_b200/csrc/sm100_ptx.cuh"]
+
+
+def traffic_from_profile(workload: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary, when it was taken on the
+    current GEMM source (else None)."""
+    p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(workload)
+    if not e or e.get("gemm_src") != src_hash(GEMM_SRC):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sharq_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait()
+
+    def summary(self):
+        if not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                rows.append(parts)
+        os.remove(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "power_w_max": max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+                if any(r[2].replace(".", "").isdigit() for r in rows) else None}
+
+
+def make_inputs(workload: str, seed: int):
+    from workloads import gaussian_weight, heavy_activations
+    M, K, N, per_row = WORKLOADS[workload]
+    rng = np.random.default_rng(seed)
+    x = heavy_activations(rng, M, K, per_row=per_row)
+    w = gaussian_weight(rng, K, N)
+    return x, w
+
+
+def cpu_baseline(workload: str, budget_s: float = 20.0, x=None, w=None):
+    """The oracle as it stands, on a bounded sample: `rows` token rows prepared and
+    multiplied by the whole (already quantised) weight. Returns (TFLOP/s, cores, sample)."""
+    from oracle import sharq as S
+    M, K, N, _ = WORKLOADS[workload]
+    if x is None:
+        x, w = make_inputs(workload, 7)
+    qw = S.quantize_weight(w.values)  # offline step, not timed
+    s_g = S.tensor_scale(x.values)
+    rows = 16
+    t_used, n_rows = 0.0, 0
+    while t_used < budget_s and n_rows < M:
+        t0 = time.perf_counter()
+        p = S.prepare(x.values[n_rows:n_rows + rows], s_g=s_g)
+        S.linear(p, qw)
+        t_used += time.perf_counter() - t0
+        n_rows += rows
+    flops = 2.0 * n_rows * N * K
+    cores = len(os.sched_getaffinity(0))
+    return flops / t_used / 1e12, cores, f"{n_rows} of {M} rows x all {N} columns, K={K}; " \
+        f"{t_used:.1f} s of CPU work (weight quantised beforehand)"
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    M, K, N, _ = WORKLOADS[args.workload]
+    x, w = make_inputs(args.workload, 7)
+    for _ in range(args.warmup):
+        pass  # the oracle has no state to warm
+    vals = []
+    budget = max(2.0, 60.0 / max(1, args.steps))
+    for _ in range(args.steps):
+        v, cores, sample = cpu_baseline(args.workload, budget, x, w)
+        vals.append(v)
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 2.0 * M * N * K / (value * 1e12) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": "nvfp4",
+                   "mask": "pair48"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import fp4_sparse_dense_b200 as sq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    M, K, N, _ = WORKLOADS[args.workload]
+    cfg = sq.Config()  # NVFP4, pair-wise 4:8, residual on
+
+    x16, w16 = make_inputs(args.workload, 1000 + rank)
+    from tests.gpu_helpers import to_device
+    n_sets = 3
+    X = [to_device(x16).to(dev) for _ in range(n_sets)]
+    W = [to_device(w16).to(dev) for _ in range(2)]
+    QW = [sq.quantize_weight(w) for w in W]
+    ACT = [sq.empty_act(M, K, cfg, dev) for _ in range(n_sets)]
+    Y = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(n_sets)]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        a = sq.prepare(X[i % n_sets], cfg, out=ACT[i % n_sets])
+        return a
+
+    for i in range(args.warmup):
+        sq.linear(step(i), QW[i % 2], out=Y[i % n_sets])
+    torch.cuda.synchronize()
+    status = sq.sharq_device_status()
+    assert status == 0, sq.sharq_status_string(status)
+
+    # per-kernel events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            a = step(i)
+            ev[i][1].record(stream)
+            sq.linear(a, QW[i % 2], out=Y[i % n_sets])
+            ev[i][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    prep_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    flops = 2.0 * M * N * K
+    value = flops * world * args.steps / (ms_max * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    xh = [X[i].cpu().pin_memory() for i in range(n_sets)]
+    yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, min(args.steps, 10))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        X[i % n_sets].copy_(xh[i % n_sets], non_blocking=True)
+        a = step(i)
+        sq.linear(a, QW[i % 2], out=Y[i % n_sets])
+        yh.copy_(Y[i % n_sets], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = flops * world * e2e_steps / (float(te.item()) * 1e-3) / 1e12
+    status = sq.sharq_device_status()
+    assert status == 0, sq.sharq_status_string(status)
+
+    if rank == 0:
+        hbm, bf16, bf16_sus, peak_src = load_peaks()
+        fp4_peak = bf16_sus * FP4_OVER_BF16
+        gemm_avg = float(np.mean(gemm_ms))
+        prep_avg = float(np.mean(prep_ms))
+        gemm_tflops = flops / (gemm_avg * 1e-3) / 1e12
+        prep_gbs = M * K * PREP_BYTES_PER_ELEM["pair48"] / (prep_avg * 1e-3) / 1e9
+        traffic = traffic_from_profile(args.workload)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": "nvfp4",
+                       "mask": "pair48", "residual": True, "out": "bf16",
+                       "l2": f"{n_sets} rotating input sets (> 126 MB L2 per step)",
+                       "parallelism": f"dp{world}"},
+            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
+                         "traffic": traffic,
+                         "peak_source": f"{peak_src}: bf16 sustained {bf16_sus} x "
+                                        f"{FP4_OVER_BF16} (nominal FP4:BF16)",
+                         "ceiling_frac": 2.0 / 3.0,
+                         "kernel": "sharq_gemm_kernel", "kernel_ms": gemm_avg},
+            "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
+                     "frac": prep_gbs / hbm,
+                     "bytes_per_elem": PREP_BYTES_PER_ELEM["pair48"],
+                     "note": "amax pass + fused prep kernel, algorithmic bytes of the prep "
+                             "kernel only"},
+            "gemm_tflops": gemm_tflops,
+            "pct_fp4_peak": 100.0 * gemm_tflops / fp4_peak,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
+                    "d2h_bytes_per_step": M * N * 2},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline and world == 1:
+            v, cores, sample = cpu_baseline(args.workload, args.cpu_budget, x16, w16)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores,
+                                    "kind": "oracle", "sample": sample}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
+    ap.add_argument("--workload", default="mlp_gate_up", choices=list(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

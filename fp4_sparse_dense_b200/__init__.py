@@ -1,0 +1,159 @@
+"""SharQ sparse-dense FP4 linear layer for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/sharq.h`` (library ``lib/libsharq.so``,
+built in-tree by ``fp4_sparse_dense_b200.build``). Every step of the path runs in the
+library's CUDA kernels; this module only marshals arguments and allocates the caller-owned
+buffers with torch. There is no CPU fallback: if the library is missing or the device is
+not an sm_100 GPU the calls raise.
+
+Low-level names mirror the C entry points (``sharq_prepare``, ``sharq_linear`` ...);
+``quantize_weight``, ``prepare`` and ``linear`` are the tensor-level conveniences.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+from ._abi import (  # noqa: F401
+    ELEM_2_4, F16, F32, BF16, MXFP4, NVFP4, PAIR_4_8, SharqError, lib, lib_path,
+    sharq_act, sharq_act_bytes, sharq_config, sharq_weight, sharq_weight_bytes, check,
+    sharq_act_sizes, sharq_weight_sizes, sharq_status_string, sharq_device_status,
+    sharq_prepare, sharq_quantize_weight, sharq_linear,
+)
+
+__all__ = [
+    "Config", "QuantWeight", "PreparedAct", "quantize_weight", "prepare", "linear",
+    "sharq_act_sizes", "sharq_weight_sizes", "sharq_prepare", "sharq_quantize_weight",
+    "sharq_linear", "sharq_device_status", "sharq_status_string", "SharqError",
+    "NVFP4", "MXFP4", "PAIR_4_8", "ELEM_2_4", "F16", "BF16", "F32",
+]
+
+
+@dataclass(frozen=True)
+class Config:
+    fmt: int = NVFP4
+    mask: int = PAIR_4_8
+    residual: bool = True
+
+    def c(self) -> sharq_config:
+        return sharq_config(self.fmt, self.mask, 1 if self.residual else 0)
+
+    @staticmethod
+    def from_names(fmt: str = "nvfp4", mask: str = "pair48", residual: bool = True) -> "Config":
+        return Config({"nvfp4": NVFP4, "mxfp4": MXFP4}[fmt],
+                      {"pair48": PAIR_4_8, "elem24": ELEM_2_4}[mask], residual)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float16:
+        return F16
+    raise TypeError(f"unsupported input dtype {t.dtype} (need bfloat16 or float16)")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+@dataclass
+class QuantWeight:
+    codes: object
+    scales_dense: object
+    scales_sparse: object
+    tensor_scale: object
+    K: int
+    N: int
+    cfg: Config
+
+    def c(self) -> sharq_weight:
+        return sharq_weight(_ptr(self.codes), _ptr(self.scales_dense), _ptr(self.scales_sparse),
+                            _ptr(self.tensor_scale), self.K, self.N, self.cfg.c())
+
+
+@dataclass
+class PreparedAct:
+    bq: object
+    bs: object
+    bm: object
+    rq: object
+    rs: object
+    tensor_scale: object
+    M: int
+    K: int
+    cfg: Config
+
+    def c(self) -> sharq_act:
+        return sharq_act(_ptr(self.bq), _ptr(self.bs), _ptr(self.bm), _ptr(self.rq), _ptr(self.rs),
+                         _ptr(self.tensor_scale), self.M, self.K, self.cfg.c())
+
+
+def _u8(n: int, device):
+    torch = _torch()
+    # 16-byte minimum so that every buffer has a valid, aligned address
+    return torch.empty(max(int(n), 16), dtype=torch.uint8, device=device)
+
+
+def empty_weight(K: int, N: int, cfg: Config, device="cuda") -> QuantWeight:
+    torch = _torch()
+    sz = sharq_weight_bytes()
+    check(sharq_weight_sizes(K, N, cfg.c(), ctypes.byref(sz)))
+    return QuantWeight(_u8(sz.codes, device), _u8(sz.scales_dense, device),
+                       _u8(sz.scales_sparse, device) if sz.scales_sparse else None,
+                       torch.zeros(4, dtype=torch.float32, device=device), K, N, cfg)
+
+
+def empty_act(M: int, K: int, cfg: Config, device="cuda") -> PreparedAct:
+    torch = _torch()
+    sz = sharq_act_bytes()
+    check(sharq_act_sizes(M, K, cfg.c(), ctypes.byref(sz)))
+    return PreparedAct(_u8(sz.bq, device), _u8(sz.bs, device), _u8(sz.bm, device),
+                       _u8(sz.rq, device) if sz.rq else None,
+                       _u8(sz.rs, device) if sz.rs else None,
+                       torch.zeros(4, dtype=torch.float32, device=device), M, K, cfg)
+
+
+def quantize_weight(W, cfg: Config = Config(), out: QuantWeight | None = None,
+                    stream=None) -> QuantWeight:
+    """W: CUDA tensor [K x N] (bf16/fp16) -> FP4 weight payload with both scale views."""
+    K, N = W.shape
+    W = W.contiguous()
+    out = out or empty_weight(K, N, cfg, W.device)
+    cw = out.c()
+    check(sharq_quantize_weight(_ptr(W), _dtype_code(W), ctypes.byref(cw), _stream(stream)))
+    return out
+
+
+def prepare(X, cfg: Config = Config(), out: PreparedAct | None = None, stream=None) -> PreparedAct:
+    """X: CUDA tensor [M x K] (bf16/fp16) -> backbone / residual FP4 operands."""
+    M, K = X.shape
+    X = X.contiguous()
+    out = out or empty_act(M, K, cfg, X.device)
+    ca = out.c()
+    check(sharq_prepare(_ptr(X), _dtype_code(X), ctypes.byref(ca), _stream(stream)))
+    return out
+
+
+def linear(act: PreparedAct, w: QuantWeight, out=None, out_dtype=None, stream=None):
+    """Y[M x N] = sparse-FP4-GEMM(backbone, W) + dense-FP4-GEMM(residual, W)."""
+    torch = _torch()
+    out_dtype = out_dtype or torch.bfloat16
+    if out is None:
+        out = torch.empty(act.M, w.N, dtype=out_dtype, device=act.bq.device)
+    code = {torch.bfloat16: BF16, torch.float32: F32}[out.dtype]
+    ca, cw = act.c(), w.c()
+    check(sharq_linear(ctypes.byref(ca), ctypes.byref(cw), _ptr(out), code, _stream(stream)))
+    return out

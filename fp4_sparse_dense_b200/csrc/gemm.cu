@@ -1,0 +1,388 @@
+// SharQ sparse + dense FP4 GEMM on sm_100a tensor cores (tcgen05, TMEM, TMA).
+//
+// SharQ page (pith.science 2606.26587), "Core claim" and abstract: the backbone goes
+// through a structured-sparse FP4 GEMM, the residual through a dense FP4 GEMM that makes
+// up for what the mask dropped and for the backbone's rounding, and both read the same
+// FP4 weight codes, each with its own view of the weight scales. Here both GEMMs are one
+// kernel: for every 256-wide K step the same weight tile in shared memory feeds two
+// structured-sparse block-scaled MMAs (backbone, 128 logical K each) and four dense
+// block-scaled MMAs (residual, 64 K each), all accumulating into one FP32 accumulator in
+// tensor memory, which one epilogue scales by alpha = s_g * s_gw and writes once.
+//
+// CTA organisation (persistent, one CTA per SM, 6 warps):
+//   warp 0      TMA producer: FP4 tiles by tensor-map loads, scales and metadata by
+//               1-D bulk copies, all completing on the stage's "full" mbarrier;
+//   warp 1      tensor-memory owner and single-thread MMA issuer: copies the stage's
+//               scales / metadata into tensor memory (tcgen05.cp) and issues the MMAs;
+//               tcgen05.commit releases the stage and, after the last K step, the
+//               accumulator;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows, scale, convert, store.
+// Tensor memory: columns [0, BN) accumulator, columns from 256 the scale factors and the
+// sparse metadata of the current K step (single-buffered: the copy and the MMAs are
+// issued by one thread and execute in issue order).
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sharq_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace sharq {
+
+constexpr int kMaxSmem = 232448;  // 227 KB opt-in dynamic shared memory per CTA
+
+template <int FMT, bool PAIR, bool RES, int BN>
+struct GemmCfg {
+  static constexpr bool NV = FMT == SHARQ_NVFP4;
+  static constexpr int GD = NV ? 16 : 32;        // dense-view scale granularity (A and W)
+  static constexpr int DCH = 256 / GD / 4;       // 512-byte scale chunks per K step (dense)
+  static constexpr bool DENSE_W = RES || !PAIR;  // any dense MMA issued
+  // bytes per stage
+  static constexpr int W_BYTES = BN * 128;
+  static constexpr int R_BYTES = RES ? 128 * 128 : 0;
+  static constexpr int B_BYTES = PAIR ? 128 * 64 : 128 * 128;
+  static constexpr int SFR_BYTES = RES ? DCH * 512 : 0;
+  static constexpr int SFB_BYTES = PAIR ? 2 * 512 : DCH * 512;
+  static constexpr int SWD_BYTES = DENSE_W ? (BN / 128) * DCH * 512 : 0;
+  static constexpr int SWS_BYTES = PAIR ? (BN / 128) * 2 * 512 : 0;
+  static constexpr int E_BYTES = PAIR ? 2048 : 0;
+  static constexpr int OFF_W = 0;
+  static constexpr int OFF_R = OFF_W + W_BYTES;
+  static constexpr int OFF_B = OFF_R + R_BYTES;
+  static constexpr int OFF_SFR = OFF_B + B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFR + SFR_BYTES;
+  static constexpr int OFF_SWD = OFF_SFB + SFB_BYTES;
+  static constexpr int OFF_SWS = OFF_SWD + SWD_BYTES;
+  static constexpr int OFF_E = OFF_SWS + SWS_BYTES;
+  static constexpr int STAGE_RAW = OFF_E + E_BYTES;
+  static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
+  static constexpr int TX = STAGE_RAW;  // every byte of the stage arrives by copy
+  static constexpr int STAGES_FIT = (kMaxSmem - 2048) / STAGE;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static constexpr int SMEM = STAGES * STAGE + 2048;  // + alignment slack and barriers
+  // tensor-memory columns
+  static constexpr int COL_SFR = 256;
+  static constexpr int COL_SFB = COL_SFR + (RES ? DCH * 4 : 0);
+  static constexpr int COL_SWD = COL_SFB + (PAIR ? 8 : DCH * 4);
+  static constexpr int COL_SWS = COL_SWD + (DENSE_W ? DCH * (BN / 32) : 0);
+  static constexpr int COL_E = COL_SWS + (PAIR ? 2 * (BN / 32) : 0);
+  static constexpr int COL_END = COL_E + (PAIR ? 4 : 0);
+  static_assert(COL_END <= 512, "tensor memory overflow");
+  static_assert(STAGES >= 2, "not enough shared memory for two stages");
+  // instruction descriptors (block-scaled kinds): E2M1 A and B, M = 128, N = BN
+  static constexpr uint32_t IDESC_BASE =
+      (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static constexpr uint32_t SCALE_FMT = NV ? 0u : (1u << 23);  // E4M3 or E8M0 scales
+};
+
+template <int FMT, bool PAIR, bool RES, int BN, bool OUT_F32>
+__global__ void __launch_bounds__(192, 1)
+    sharq_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
+                      const __grid_constant__ CUtensorMap tm_b,
+                      const __grid_constant__ CUtensorMap tm_r, const GemmParams p) {
+  using C = GemmCfg<FMT, PAIR, RES, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ctrl = smem + C::STAGES * C::STAGE;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* empty_bar = full_bar + C::STAGES;
+  uint64_t* tfull_bar = empty_bar + C::STAGES;
+  uint64_t* tempty_bar = tfull_bar + 1;
+  uint64_t* drain_bar = tempty_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int KT = p.K / 256;
+  const int tiles = p.tiles_m * p.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      ptx::mbar_init(ptx::smem_u32(full_bar + s), 1);
+      ptx::mbar_init(ptx::smem_u32(empty_bar + s), 1);
+    }
+    ptx::mbar_init(ptx::smem_u32(tfull_bar), 1);
+    ptx::mbar_init(ptx::smem_u32(tempty_bar), 128);
+    ptx::mbar_init(ptx::smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tensormap(&tm_w);
+    ptx::prefetch_tensormap(&tm_b);
+    if (RES) ptx::prefetch_tensormap(&tm_r);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint64_t limit = p.timeout_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (ptx::elect_one()) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int mb = t % p.tiles_m, nb = t / p.tiles_m;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!ptx::mbar_wait(ptx::smem_u32(empty_bar + s), ph ^ 1u, abort_flag, limit)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = ptx::smem_u32(full_bar + s);
+          ptx::mbar_arrive_expect_tx(fb, C::TX);
+          uint8_t* st = smem + s * C::STAGE;
+          ptx::tma_load_2d(ptx::smem_u32(st + C::OFF_W), &tm_w, kt * 128, nb * BN, fb);
+          if (RES) ptx::tma_load_2d(ptx::smem_u32(st + C::OFF_R), &tm_r, kt * 128, mb * 128, fb);
+          ptx::tma_load_2d(ptx::smem_u32(st + C::OFF_B), &tm_b, kt * (PAIR ? 64 : 128), mb * 128,
+                           fb);
+          if (RES) {
+            const uint8_t* src = p.rs + (size_t(mb) * (p.K / C::GD / 4) + size_t(kt) * C::DCH) * 512;
+            ptx::bulk_load(ptx::smem_u32(st + C::OFF_SFR), src, C::SFR_BYTES, fb);
+          }
+          if (PAIR) {
+            const uint8_t* src = p.bs + (size_t(mb) * (p.K / 32 / 4) + size_t(kt) * 2) * 512;
+            ptx::bulk_load(ptx::smem_u32(st + C::OFF_SFB), src, C::SFB_BYTES, fb);
+            const uint8_t* e = p.bm + size_t(kt) * p.Mp * 16 + size_t(mb) * 2048;
+            ptx::bulk_load(ptx::smem_u32(st + C::OFF_E), e, 2048, fb);
+            for (int rb = 0; rb < BN / 128; ++rb) {
+              const uint8_t* w =
+                  p.wss + (size_t(nb * (BN / 128) + rb) * (p.K / 32 / 4) + size_t(kt) * 2) * 512;
+              ptx::bulk_load(ptx::smem_u32(st + C::OFF_SWS + rb * 1024), w, 1024, fb);
+            }
+          } else {
+            const uint8_t* src = p.bs + (size_t(mb) * (p.K / C::GD / 4) + size_t(kt) * C::DCH) * 512;
+            ptx::bulk_load(ptx::smem_u32(st + C::OFF_SFB), src, C::SFB_BYTES, fb);
+          }
+          if (C::DENSE_W) {
+            for (int rb = 0; rb < BN / 128; ++rb) {
+              const uint8_t* w = p.wsd + (size_t(nb * (BN / 128) + rb) * (p.K / C::GD / 4) +
+                                          size_t(kt) * C::DCH) * 512;
+              ptx::bulk_load(ptx::smem_u32(st + C::OFF_SWD + rb * C::DCH * 512), w, C::DCH * 512,
+                             fb);
+            }
+          }
+          if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) atomicExch(p.status, unsigned(SHARQ_ERR_TIMEOUT));
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (ptx::elect_one()) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int tcount = 0;
+      const uint32_t idesc_d = C::IDESC_BASE | C::SCALE_FMT;
+      const uint32_t idesc_s = C::IDESC_BASE | C::SCALE_FMT | (1u << 2);
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tcount) {
+        if (tcount > 0) {
+          if (!ptx::mbar_wait(ptx::smem_u32(tempty_bar), uint32_t(tcount - 1) & 1u, abort_flag,
+                              limit)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+        }
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!ptx::mbar_wait(ptx::smem_u32(full_bar + s), ph, abort_flag, limit)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t st = ptx::smem_u32(smem + s * C::STAGE);
+          // ---- scale factors and metadata of this K step into tensor memory
+          if (PAIR) {
+            ptx::tmem_cp_128x128b(tbase + C::COL_E, ptx::smem_desc(st + C::OFF_E, 16, 128, 0));
+            for (int j = 0; j < 2; ++j) {
+              ptx::tmem_cp_32x128b_x4(tbase + C::COL_SFB + 4 * j,
+                                      ptx::smem_desc(st + C::OFF_SFB + 512 * j, 16, 128, 0));
+              for (int rb = 0; rb < BN / 128; ++rb)
+                ptx::tmem_cp_32x128b_x4(
+                    tbase + C::COL_SWS + j * (BN / 32) + 4 * rb,
+                    ptx::smem_desc(st + C::OFF_SWS + (rb * 2 + j) * 512, 16, 128, 0));
+            }
+          } else {
+            for (int c = 0; c < C::DCH; ++c)
+              ptx::tmem_cp_32x128b_x4(tbase + C::COL_SFB + 4 * c,
+                                      ptx::smem_desc(st + C::OFF_SFB + 512 * c, 16, 128, 0));
+          }
+          if (RES) {
+            for (int c = 0; c < C::DCH; ++c)
+              ptx::tmem_cp_32x128b_x4(tbase + C::COL_SFR + 4 * c,
+                                      ptx::smem_desc(st + C::OFF_SFR + 512 * c, 16, 128, 0));
+          }
+          if (C::DENSE_W) {
+            for (int c = 0; c < C::DCH; ++c)
+              for (int rb = 0; rb < BN / 128; ++rb)
+                ptx::tmem_cp_32x128b_x4(
+                    tbase + C::COL_SWD + c * (BN / 32) + 4 * rb,
+                    ptx::smem_desc(st + C::OFF_SWD + (rb * C::DCH + c) * 512, 16, 128, 0));
+          }
+          // ---- MMAs: backbone then residual, one accumulator
+          uint32_t acc = kt > 0 ? 1u : 0u;
+          if (PAIR) {
+            for (int j = 0; j < 2; ++j) {
+              const uint64_t a = ptx::smem_desc(st + C::OFF_B + 32 * j, 16, 512, 4);
+              const uint64_t b = ptx::smem_desc(st + C::OFF_W + 64 * j, 16, 1024, 2);
+              ptx::mma_sp_nvf4(tbase, a, b, tbase + C::COL_E + 2 * j, idesc_s,
+                               tbase + C::COL_SFB + 4 * j, tbase + C::COL_SWS + j * (BN / 32), acc);
+              acc = 1u;
+            }
+          } else {
+            for (int i = 0; i < 4; ++i) {
+              const uint64_t a = ptx::smem_desc(st + C::OFF_B + 32 * i, 16, 1024, 2);
+              const uint64_t b = ptx::smem_desc(st + C::OFF_W + 32 * i, 16, 1024, 2);
+              if (C::NV) {
+                ptx::mma_nvf4(tbase, a, b, idesc_d, tbase + C::COL_SFB + 4 * i,
+                              tbase + C::COL_SWD + i * (BN / 32), acc);
+              } else {
+                const uint32_t id = 2u * uint32_t(i & 1);
+                ptx::mma_mxf4(tbase, a, b, idesc_d | (id << 29) | (id << 4),
+                              (tbase + C::COL_SFB + 4 * (i >> 1)) | (id << 30),
+                              (tbase + C::COL_SWD + (i >> 1) * (BN / 32)) | (id << 30), acc);
+              }
+              acc = 1u;
+            }
+          }
+          if (RES) {
+            for (int i = 0; i < 4; ++i) {
+              const uint64_t a = ptx::smem_desc(st + C::OFF_R + 32 * i, 16, 1024, 2);
+              const uint64_t b = ptx::smem_desc(st + C::OFF_W + 32 * i, 16, 1024, 2);
+              if (C::NV) {
+                ptx::mma_nvf4(tbase, a, b, idesc_d, tbase + C::COL_SFR + 4 * i,
+                              tbase + C::COL_SWD + i * (BN / 32), 1u);
+              } else {
+                const uint32_t id = 2u * uint32_t(i & 1);
+                ptx::mma_mxf4(tbase, a, b, idesc_d | (id << 29) | (id << 4),
+                              (tbase + C::COL_SFR + 4 * (i >> 1)) | (id << 30),
+                              (tbase + C::COL_SWD + (i >> 1) * (BN / 32)) | (id << 30), 1u);
+              }
+            }
+          }
+          ptx::mma_commit(ptx::smem_u32(empty_bar + s));
+          if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        ptx::mma_commit(ptx::smem_u32(tfull_bar));
+      }
+      // drain: every tcgen05 operation issued above has finished once this arrives
+      ptx::mma_commit(ptx::smem_u32(drain_bar));
+      if (!ptx::mbar_wait(ptx::smem_u32(drain_bar), 0, abort_flag, limit)) ok = false;
+      if (!ok) atomicExch(p.status, unsigned(SHARQ_ERR_TIMEOUT));
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // tensor-memory lane quarter this warp may access
+    const float alpha = __fmul_rn(p.act_ts[0], p.w_ts[0]);
+    int tcount = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
+      const int mb = t % p.tiles_m, nb = t / p.tiles_m;
+      if (!ptx::mbar_wait(ptx::smem_u32(tfull_bar), uint32_t(tcount) & 1u, abort_flag, limit)) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      const int row = mb * 128 + quarter * 32 + lane;
+      const uint32_t taddr = tbase + (uint32_t(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
+        ptx::tmem_ld_wait();
+        if (row < p.M) {
+          const size_t off = size_t(row) * p.N + size_t(nb) * BN + c * 32;
+          if (OUT_F32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + off);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__fmul_rn(__uint_as_float(v[4 * i]), alpha),
+                                   __fmul_rn(__uint_as_float(v[4 * i + 1]), alpha),
+                                   __fmul_rn(__uint_as_float(v[4 * i + 2]), alpha),
+                                   __fmul_rn(__uint_as_float(v[4 * i + 3]), alpha));
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + off);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat162 b2 =
+                    __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[8 * i + 2 * h]), alpha),
+                                          __fmul_rn(__uint_as_float(v[8 * i + 2 * h + 1]), alpha));
+                w4[h] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              dst[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_u32(tempty_bar));
+    }
+    if (!ok && lane == 0) atomicExch(p.status, unsigned(SHARQ_ERR_TIMEOUT));
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tbase, 512);
+  }
+}
+
+template <int FMT, bool PAIR, bool RES, int BN, bool OUT_F32>
+static cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, int num_sms, cudaStream_t st) {
+  using C = GemmCfg<FMT, PAIR, RES, BN>;
+  auto kern = sharq_gemm_kernel<FMT, PAIR, RES, BN, OUT_F32>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  kern<<<grid, 192, C::SMEM, st>>>(m.w, m.b, m.r, p);
+  return cudaGetLastError();
+}
+
+template <int FMT, bool PAIR, bool RES, int BN>
+static cudaError_t launch_o(const GemmMaps& m, const GemmParams& p, bool f32, int n, cudaStream_t st) {
+  return f32 ? launch_t<FMT, PAIR, RES, BN, true>(m, p, n, st)
+             : launch_t<FMT, PAIR, RES, BN, false>(m, p, n, st);
+}
+
+template <int FMT, bool PAIR, bool RES>
+static cudaError_t launch_n(const GemmMaps& m, const GemmParams& p, bool f32, int n, cudaStream_t st) {
+  return (p.N % 256 == 0) ? launch_o<FMT, PAIR, RES, 256>(m, p, f32, n, st)
+                          : launch_o<FMT, PAIR, RES, 128>(m, p, f32, n, st);
+}
+
+template <int FMT, bool PAIR>
+static cudaError_t launch_r(const GemmMaps& m, const GemmParams& p, bool res, bool f32, int n,
+                            cudaStream_t st) {
+  return res ? launch_n<FMT, PAIR, true>(m, p, f32, n, st)
+             : launch_n<FMT, PAIR, false>(m, p, f32, n, st);
+}
+
+template <int FMT>
+static cudaError_t launch_m(const GemmMaps& m, const GemmParams& p, int mask, bool res, bool f32,
+                            int n, cudaStream_t st) {
+  return mask == SHARQ_MASK_PAIR_4_8 ? launch_r<FMT, true>(m, p, res, f32, n, st)
+                                     : launch_r<FMT, false>(m, p, res, f32, n, st);
+}
+
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int mask,
+                        bool residual, bool out_f32, int num_sms, cudaStream_t st) {
+  return fmt == SHARQ_NVFP4 ? launch_m<SHARQ_NVFP4>(maps, p, mask, residual, out_f32, num_sms, st)
+                            : launch_m<SHARQ_MXFP4>(maps, p, mask, residual, out_f32, num_sms, st);
+}
+
+}  // namespace sharq

@@ -1,0 +1,342 @@
+// C ABI of the SharQ library: argument checks, buffer-size queries, TMA descriptor
+// construction and the launches of the preparation, weight-quantisation and GEMM
+// kernels. See include/sharq.h for the contract of every entry point.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sharq_internal.h"
+
+namespace sharq {
+
+// Written by kernels that give up on a bounded wait; read and cleared by
+// sharq_device_status(). One word per device (the array is per device image).
+__device__ unsigned int g_status_word;
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per mbarrier wait
+
+struct DeviceInfo {
+  bool ok = false;
+  int num_sms = 0;
+  unsigned int* status = nullptr;
+};
+
+std::mutex g_mu;
+std::unordered_map<int, DeviceInfo> g_dev;
+
+sharq_status device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SHARQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_dev.find(dev);
+  if (it != g_dev.end()) {
+    *out = it->second;
+    return out->ok ? SHARQ_OK : SHARQ_ERR_ARCH;
+  }
+  DeviceInfo d;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return SHARQ_ERR_CUDA;
+  d.ok = (major == 10 && minor == 0);
+  if (d.ok) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return SHARQ_ERR_CUDA;
+    d.status = static_cast<unsigned int*>(p);
+  }
+  g_dev[dev] = d;
+  *out = d;
+  return d.ok ? SHARQ_OK : SHARQ_ERR_ARCH;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sharq_status check_cfg(sharq_config c) {
+  if (c.fmt != SHARQ_NVFP4 && c.fmt != SHARQ_MXFP4) return SHARQ_ERR_INVALID_ARG;
+  if (c.mask != SHARQ_MASK_PAIR_4_8 && c.mask != SHARQ_MASK_ELEM_2_4) return SHARQ_ERR_INVALID_ARG;
+  if (c.residual != 0 && c.residual != 1) return SHARQ_ERR_INVALID_ARG;
+  return SHARQ_OK;
+}
+
+size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+size_t tiled_bytes(size_t rows, size_t cols) { return round_up(rows, 128) * round_up(cols, 4); }
+
+sharq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA; }
+
+// ------------------------------------------------------------------ TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct MapKey {
+  const void* ptr;
+  uint64_t inner, rows;
+  uint32_t box_inner, box_rows, swz;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && inner == o.inner && rows == o.rows && box_inner == o.box_inner &&
+           box_rows == o.box_rows && swz == o.swz;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    size_t h = reinterpret_cast<size_t>(k.ptr);
+    h ^= (k.inner * 0x9E3779B97F4A7C15ull) + (h << 6) + (h >> 2);
+    h ^= (k.rows * 0xC2B2AE3D27D4EB4Full) + (h << 6) + (h >> 2);
+    h ^= (uint64_t(k.box_inner) << 32 | uint64_t(k.box_rows) << 8 | k.swz) + (h << 6) + (h >> 2);
+    return h;
+  }
+};
+std::mutex g_map_mu;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
+
+// 2-D byte matrix [rows][inner] (row pitch = inner), box [box_rows][box_inner]
+sharq_status make_map(CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t rows,
+                      uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  MapKey key{ptr, inner, rows, box_inner, box_rows, uint32_t(swz)};
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *out = it->second;
+      return SHARQ_OK;
+    }
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return SHARQ_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return SHARQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  if (g_maps.size() > 4096) g_maps.clear();
+  g_maps[key] = *out;
+  return SHARQ_OK;
+}
+
+sharq_status act_sizes(int32_t M, int32_t K, sharq_config c, sharq_act_bytes* o) {
+  if (!o || M < 1 || K < 256 || K % 256 != 0) return SHARQ_ERR_INVALID_ARG;
+  sharq_status s = check_cfg(c);
+  if (s != SHARQ_OK) return s;
+  const bool pair = c.mask == SHARQ_MASK_PAIR_4_8;
+  const size_t m = size_t(M), k = size_t(K);
+  o->bq = pair ? m * k / 4 : m * k / 2;
+  o->bs = tiled_bytes(m, k / size_t(backbone_block(c.fmt, c.mask)));
+  o->bm = pair ? round_up(m, 128) * k / 16 : m * k / 8;
+  o->rq = c.residual ? m * k / 2 : 0;
+  o->rs = c.residual ? tiled_bytes(m, k / size_t(residual_block(c.fmt))) : 0;
+  return SHARQ_OK;
+}
+
+sharq_status weight_sizes(int32_t K, int32_t N, sharq_config c, sharq_weight_bytes* o) {
+  if (!o || K < 256 || K % 256 != 0 || N < 128 || N % 128 != 0) return SHARQ_ERR_INVALID_ARG;
+  sharq_status s = check_cfg(c);
+  if (s != SHARQ_OK) return s;
+  const size_t k = size_t(K), n = size_t(N);
+  o->codes = n * k / 2;
+  o->scales_dense = tiled_bytes(n, k / size_t(dense_view_block(c.fmt)));
+  o->scales_sparse = c.mask == SHARQ_MASK_PAIR_4_8 ? tiled_bytes(n, k / 32) : 0;
+  return SHARQ_OK;
+}
+
+}  // namespace
+}  // namespace sharq
+
+using namespace sharq;
+
+extern "C" {
+
+const char* sharq_status_string(sharq_status s) {
+  switch (s) {
+    case SHARQ_OK: return "SHARQ_OK";
+    case SHARQ_ERR_INVALID_ARG: return "SHARQ_ERR_INVALID_ARG";
+    case SHARQ_ERR_UNSUPPORTED: return "SHARQ_ERR_UNSUPPORTED";
+    case SHARQ_ERR_MISALIGNED: return "SHARQ_ERR_MISALIGNED";
+    case SHARQ_ERR_CUDA: return "SHARQ_ERR_CUDA";
+    case SHARQ_ERR_TIMEOUT: return "SHARQ_ERR_TIMEOUT";
+    case SHARQ_ERR_ARCH: return "SHARQ_ERR_ARCH";
+  }
+  return "SHARQ_ERR_UNKNOWN";
+}
+
+sharq_status sharq_act_sizes(int32_t M, int32_t K, sharq_config cfg, sharq_act_bytes* out) {
+  return act_sizes(M, K, cfg, out);
+}
+
+sharq_status sharq_weight_sizes(int32_t K, int32_t N, sharq_config cfg, sharq_weight_bytes* out) {
+  return weight_sizes(K, N, cfg, out);
+}
+
+sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, const sharq_weight* w,
+                                   void* stream) {
+  if (!W || !w) return SHARQ_ERR_INVALID_ARG;
+  if (dtype != SHARQ_F16 && dtype != SHARQ_BF16) return SHARQ_ERR_INVALID_ARG;
+  sharq_weight_bytes sz;
+  sharq_status s = weight_sizes(w->K, w->N, w->cfg, &sz);
+  if (s != SHARQ_OK) return s;
+  const bool pair = w->cfg.mask == SHARQ_MASK_PAIR_4_8;
+  if (!w->codes || !w->scales_dense || !w->tensor_scale || (pair && !w->scales_sparse))
+    return SHARQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(w->codes) || !aligned16(w->scales_dense) ||
+      !aligned16(w->tensor_scale) || (pair && !aligned16(w->scales_sparse)))
+    return SHARQ_ERR_MISALIGNED;
+  DeviceInfo d;
+  if ((s = device_info(&d)) != SHARQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == SHARQ_BF16;
+  if (w->cfg.fmt == SHARQ_NVFP4) {
+    if (cudaMemsetAsync(w->tensor_scale + 1, 0, sizeof(float), st) != cudaSuccess)
+      return SHARQ_ERR_CUDA;
+    s = from_cuda(launch_amax(W, bf16, size_t(w->K) * size_t(w->N),
+                              reinterpret_cast<unsigned int*>(w->tensor_scale + 1), d.num_sms, st));
+    if (s != SHARQ_OK) return s;
+  }
+  WeightQuantParams p;
+  p.W = W;
+  p.codes = static_cast<uint8_t*>(w->codes);
+  p.scales_dense = static_cast<uint8_t*>(w->scales_dense);
+  p.scales_sparse = static_cast<uint8_t*>(w->scales_sparse);
+  p.tensor_scale = w->tensor_scale;
+  p.K = w->K;
+  p.N = w->N;
+  return from_cuda(launch_weight_quant(p, bf16, w->cfg.fmt, w->cfg.mask, st));
+}
+
+sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* a, void* stream) {
+  if (!X || !a) return SHARQ_ERR_INVALID_ARG;
+  if (dtype != SHARQ_F16 && dtype != SHARQ_BF16) return SHARQ_ERR_INVALID_ARG;
+  sharq_act_bytes sz;
+  sharq_status s = act_sizes(a->M, a->K, a->cfg, &sz);
+  if (s != SHARQ_OK) return s;
+  const bool res = a->cfg.residual == 1;
+  if (!a->bq || !a->bs || !a->bm || !a->tensor_scale || (res && (!a->rq || !a->rs)))
+    return SHARQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(a->bq) || !aligned16(a->bs) || !aligned16(a->bm) ||
+      !aligned16(a->tensor_scale) || (res && (!aligned16(a->rq) || !aligned16(a->rs))))
+    return SHARQ_ERR_MISALIGNED;
+  DeviceInfo d;
+  if ((s = device_info(&d)) != SHARQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == SHARQ_BF16;
+  if (a->cfg.fmt == SHARQ_NVFP4) {
+    if (cudaMemsetAsync(a->tensor_scale + 1, 0, sizeof(float), st) != cudaSuccess)
+      return SHARQ_ERR_CUDA;
+    s = from_cuda(launch_amax(X, bf16, size_t(a->M) * size_t(a->K),
+                              reinterpret_cast<unsigned int*>(a->tensor_scale + 1), d.num_sms, st));
+    if (s != SHARQ_OK) return s;
+  }
+  PrepParams p;
+  p.X = X;
+  p.bq = a->bq;
+  p.bs = a->bs;
+  p.bm = a->bm;
+  p.rq = a->rq;
+  p.rs = a->rs;
+  p.tensor_scale = a->tensor_scale;
+  p.amax = a->tensor_scale + 1;
+  p.M = a->M;
+  p.K = a->K;
+  p.Mp = int(round_up(size_t(a->M), 128));
+  return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, st));
+}
+
+sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sharq_dtype y_dtype,
+                          void* stream) {
+  if (!a || !w || !Y) return SHARQ_ERR_INVALID_ARG;
+  if (y_dtype != SHARQ_BF16 && y_dtype != SHARQ_F32) return SHARQ_ERR_INVALID_ARG;
+  if (std::memcmp(&a->cfg, &w->cfg, sizeof(sharq_config)) != 0 || a->K != w->K)
+    return SHARQ_ERR_INVALID_ARG;
+  sharq_act_bytes asz;
+  sharq_weight_bytes wsz;
+  sharq_status s = act_sizes(a->M, a->K, a->cfg, &asz);
+  if (s != SHARQ_OK) return s;
+  if ((s = weight_sizes(w->K, w->N, w->cfg, &wsz)) != SHARQ_OK) return s;
+  const bool res = a->cfg.residual == 1, pair = a->cfg.mask == SHARQ_MASK_PAIR_4_8;
+  if (!a->bq || !a->bs || !a->tensor_scale || (pair && !a->bm) || (res && (!a->rq || !a->rs)) ||
+      !w->codes || !w->tensor_scale || ((res || !pair) && !w->scales_dense) ||
+      (pair && !w->scales_sparse))
+    return SHARQ_ERR_INVALID_ARG;
+  if (!aligned16(Y) || !aligned16(a->bq) || !aligned16(a->bs) || !aligned16(a->bm) ||
+      !aligned16(a->rq) || !aligned16(a->rs) || !aligned16(w->codes) ||
+      !aligned16(w->scales_dense) || !aligned16(w->scales_sparse))
+    return SHARQ_ERR_MISALIGNED;
+  DeviceInfo d;
+  if ((s = device_info(&d)) != SHARQ_OK) return s;
+  const int M = a->M, K = a->K, N = w->N;
+  const int BN = (N % 256 == 0) ? 256 : 128;
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if ((s = make_map(&maps.w, w->codes, uint64_t(K) / 2, uint64_t(N), 128, uint32_t(BN),
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != SHARQ_OK)
+    return s;
+  if (pair)
+    s = make_map(&maps.b, a->bq, uint64_t(K) / 4, uint64_t(M), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+  else
+    s = make_map(&maps.b, a->bq, uint64_t(K) / 2, uint64_t(M), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SHARQ_OK) return s;
+  if (res && (s = make_map(&maps.r, a->rq, uint64_t(K) / 2, uint64_t(M), 128, 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != SHARQ_OK)
+    return s;
+  if (!res) maps.r = maps.b;
+  GemmParams p;
+  p.bs = static_cast<const uint8_t*>(a->bs);
+  p.bm = static_cast<const uint8_t*>(a->bm);
+  p.rs = static_cast<const uint8_t*>(a->rs);
+  p.wsd = static_cast<const uint8_t*>(w->scales_dense);
+  p.wss = static_cast<const uint8_t*>(w->scales_sparse);
+  p.act_ts = a->tensor_scale;
+  p.w_ts = w->tensor_scale;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.Mp = int(round_up(size_t(M), 128));
+  p.tiles_m = (M + 127) / 128;
+  p.tiles_n = N / BN;
+  p.status = d.status;
+  p.timeout_ns = kWaitLimitNs;
+  return from_cuda(launch_gemm(maps, p, a->cfg.fmt, a->cfg.mask, res, y_dtype == SHARQ_F32,
+                               d.num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+sharq_status sharq_device_status(void) {
+  DeviceInfo d;
+  sharq_status s = device_info(&d);
+  if (s != SHARQ_OK) return s;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SHARQ_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, d.status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SHARQ_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpy(d.status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+    return SHARQ_ERR_CUDA;
+  return v == 0 ? SHARQ_OK : static_cast<sharq_status>(v);
+}
+
+}  // extern "C"

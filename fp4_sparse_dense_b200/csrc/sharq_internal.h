@@ -1,0 +1,73 @@
+// Internal declarations shared by the SharQ CUDA translation units (not part of the ABI).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/sharq.h"
+
+namespace sharq {
+
+struct PrepParams {
+  const void* X;        // [M][K] 16-bit
+  void* bq;
+  void* bs;
+  void* bm;
+  void* rq;
+  void* rs;
+  float* tensor_scale;  // [0] = s_g (written), [1] = amax (NVFP4, read)
+  const float* amax;    // = tensor_scale + 1
+  int M, K, Mp;
+};
+
+struct WeightQuantParams {
+  const void* W;           // [K][N] 16-bit
+  uint8_t* codes;          // [N][K/2]
+  uint8_t* scales_dense;   // tiled N x K/GD
+  uint8_t* scales_sparse;  // tiled N x K/32 (pair mask) or null
+  float* tensor_scale;     // [0] = s_gw (written), [1] = amax (NVFP4, read)
+  int K, N;
+};
+
+struct GemmParams {
+  const uint8_t* bs;   // backbone scales (tiled)
+  const uint8_t* bm;   // pair metadata
+  const uint8_t* rs;   // residual scales (tiled)
+  const uint8_t* wsd;  // weight scales, dense view
+  const uint8_t* wss;  // weight scales, sparse view
+  const float* act_ts;
+  const float* w_ts;
+  void* Y;
+  int M, N, K, Mp;
+  int tiles_m, tiles_n;
+  unsigned int* status;
+  unsigned long long timeout_ns;
+};
+
+cudaError_t launch_amax(const void* X, bool bf16, size_t n_elems, unsigned int* amax_bits,
+                        int num_sms, cudaStream_t st);
+cudaError_t launch_prep(const PrepParams& p, bool bf16, int fmt, int mask, bool residual,
+                        cudaStream_t st);
+cudaError_t launch_weight_quant(const WeightQuantParams& p, bool bf16, int fmt, int mask,
+                                cudaStream_t st);
+
+// maps for the three FP4 operands, built by the host side
+struct GemmMaps {
+  CUtensorMap w, b, r;
+};
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int mask,
+                        bool residual, bool out_f32, int num_sms, cudaStream_t st);
+
+// block sizes along K
+inline int residual_block(int fmt) { return fmt == SHARQ_NVFP4 ? 16 : 32; }
+inline int backbone_block(int fmt, int mask) {
+  return mask == SHARQ_MASK_PAIR_4_8 ? 32 : residual_block(fmt);
+}
+inline int weight_block(int fmt, int mask) {
+  if (fmt == SHARQ_MXFP4) return 32;
+  return mask == SHARQ_MASK_PAIR_4_8 ? 32 : 16;
+}
+inline int dense_view_block(int fmt) { return fmt == SHARQ_NVFP4 ? 16 : 32; }
+
+}  // namespace sharq

@@ -1,0 +1,162 @@
+/*
+ * sharq.h - C ABI of the SharQ sparse-dense FP4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the one stated on the SharQ page ("SharQ: Bridging Activation
+ * Sparsity and FP4 Quantization for LLM Inference", pith.science 2606.26587, "Core
+ * claim" and arXiv abstract): for each activation tensor an input-adaptive N:M mask
+ * extracts an outlier-dominated sparse backbone, the backbone is quantised to FP4, a
+ * dense residual is defined against the quantised backbone and quantised to FP4 with its
+ * own scales, and Y = sparse-FP4-GEMM(backbone, W) + dense-FP4-GEMM(residual, W), the two
+ * GEMMs sharing one FP4 weight payload with path-specific scale views.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor arguments are DEVICE pointers into memory the caller owns. The library
+ *   never allocates or frees device memory and keeps no pointer after a call returns,
+ *   except a small host-side cache of TMA descriptors keyed by (pointer, shape).
+ * - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *   stream) and the call returns without synchronising, except sharq_device_status().
+ * - Every device pointer must be 16-byte aligned (TMA / 128-bit access); a misaligned
+ *   pointer returns SHARQ_ERR_MISALIGNED before anything is enqueued.
+ * - Shapes: K % 256 == 0, N % 128 == 0, M >= 1 (no upper bound other than int32 sizes).
+ * - Errors are returned by value; no call aborts the process. A CUDA launch error is
+ *   reported as SHARQ_ERR_CUDA. A kernel that gives up on a bounded wait records
+ *   SHARQ_ERR_TIMEOUT in a device status word read back by sharq_device_status().
+ * - The library needs an sm_100 device (B200); on anything else the compute calls return
+ *   SHARQ_ERR_ARCH. The size queries and sharq_status_string need no GPU.
+ */
+#ifndef SHARQ_H
+#define SHARQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SHARQ_API __attribute__((visibility("default")))
+#else
+#define SHARQ_API
+#endif
+
+typedef enum {
+  SHARQ_OK = 0,
+  SHARQ_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, mismatched configs */
+  SHARQ_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+  SHARQ_ERR_MISALIGNED = 3,   /* a device pointer is not 16-byte aligned */
+  SHARQ_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  SHARQ_ERR_TIMEOUT = 5,      /* a kernel hit its bounded-wait limit and exited */
+  SHARQ_ERR_ARCH = 6          /* the current device is not sm_100 */
+} sharq_status;
+
+/* FP4 encodings. NVFP4: E2M1 codes, E4M3 block scales, FP32 tensor scale.
+ * MXFP4 (OCP MX): E2M1 codes, E8M0 block scales, no tensor scale. */
+typedef enum { SHARQ_NVFP4 = 0, SHARQ_MXFP4 = 1 } sharq_format;
+
+/* Backbone masks along K. PAIR_4_8: in every 8 consecutive K elements keep 2 of the 4
+ * adjacent pairs (the structured sparsity of the sm_100a sparse FP4 MMA); pairs ranked by
+ * (max |x|, then min |x|), ties to the lower pair. ELEM_2_4: in every 4 keep the 2 largest
+ * |x|, ties to the lower index; the backbone is then stored zero-filled and runs through
+ * the dense MMA (sm_100a has no element-wise 2:4 pattern for block-scaled FP4). */
+typedef enum { SHARQ_MASK_PAIR_4_8 = 0, SHARQ_MASK_ELEM_2_4 = 1 } sharq_mask;
+
+typedef enum { SHARQ_F16 = 0, SHARQ_BF16 = 1, SHARQ_F32 = 2 } sharq_dtype;
+
+typedef struct {
+  int32_t fmt;      /* sharq_format */
+  int32_t mask;     /* sharq_mask */
+  int32_t residual; /* 1: backbone + residual (the method); 0: backbone only */
+} sharq_config;
+
+/* Block sizes along K (logical positions per scale), fixed by the MMA consuming them:
+ *   residual:  16 (NVFP4) | 32 (MXFP4)
+ *   backbone:  32 for PAIR_4_8 (16 kept values); the residual's size for ELEM_2_4
+ *   weight:    32 for PAIR_4_8 or MXFP4; 16 for NVFP4 + ELEM_2_4
+ *
+ * Byte layouts (all row-major in the sense given):
+ *   FP4 codes:  two per byte, even K index in the low nibble, rows K-major.
+ *   Scales:     one byte per (row, block); rows grouped by 128 and block columns by 4;
+ *               each 128x4 tile is a 512-byte chunk where (r, c) sits at
+ *               (r%32)*16 + ((r/32)%4)*4 + c%4; chunks run along the columns first,
+ *               then along the 128-row groups. Rows padded to 128, columns to 4.
+ *   PAIR metadata: one nibble per 8 logical K, i0 | i1<<2 (kept pair indices i0 < i1).
+ *               Per 256 logical K, rows padded to 128 are stored one after another,
+ *               16 bytes each (lower group in the low nibble); the 256-K slices follow
+ *               each other. Padding rows hold 0x44 (pairs 0 and 1).
+ *   ELEM metadata: one nibble per 4 K (element indices), row-major, K/8 bytes per row.
+ */
+
+/* Quantised weight. Filled by sharq_quantize_weight; the caller allocates the buffers
+ * with the sizes from sharq_weight_sizes and keeps them for every later sharq_linear. */
+typedef struct {
+  void* codes;         /* [N][K/2] bytes: W^T K-major, E2M1 */
+  void* scales_dense;  /* tiled scales, N x K/16 (NVFP4) or N x K/32 (MXFP4): the dense
+                          MMA's view */
+  void* scales_sparse; /* tiled scales, N x K/32: the sparse MMA's view (PAIR_4_8 only,
+                          else unused and may be NULL) */
+  float* tensor_scale; /* 2 floats: [0] s_gw = amax|W| / 2688 (NVFP4) or 1.0 (MXFP4);
+                          [1] amax|W| (NVFP4; written by the first pass) */
+  int32_t K, N;
+  sharq_config cfg;
+} sharq_weight;
+
+/* Prepared activations. Filled by sharq_prepare from X[M x K]. */
+typedef struct {
+  void* bq;            /* backbone codes: [M][K/4] bytes (PAIR, compressed) or
+                          [M][K/2] (ELEM, zero-filled) */
+  void* bs;            /* backbone scales, tiled, M x K/backbone_block */
+  void* bm;            /* metadata: PAIR layout (M_pad*K/16 bytes) or ELEM (M*K/8) */
+  void* rq;            /* residual codes [M][K/2] (unused when residual == 0) */
+  void* rs;            /* residual scales, tiled, M x K/residual_block */
+  float* tensor_scale; /* 2 floats: [0] s_g = amax|X| / 2688 (NVFP4) or 1.0 (MXFP4);
+                          [1] amax|X| (NVFP4; written by the first pass) */
+  int32_t M, K;
+  sharq_config cfg;
+} sharq_act;
+
+typedef struct { size_t bq, bs, bm, rq, rs; } sharq_act_bytes;
+typedef struct { size_t codes, scales_dense, scales_sparse; } sharq_weight_bytes;
+
+/* Byte sizes of the buffers of a sharq_act for X[M x K] under cfg. No GPU needed.
+ * Errors: INVALID_ARG (bad shape/config or out == NULL). */
+SHARQ_API sharq_status sharq_act_sizes(int32_t M, int32_t K, sharq_config cfg, sharq_act_bytes* out);
+
+/* Byte sizes of the buffers of a sharq_weight for W[K x N] under cfg. No GPU needed. */
+SHARQ_API sharq_status sharq_weight_sizes(int32_t K, int32_t N, sharq_config cfg, sharq_weight_bytes* out);
+
+/* Offline weight quantisation (SharQ page, abstract: one FP4 weight payload serves both
+ * GEMMs, each with its own view of the scales). W: device pointer to W[K x N] row-major
+ * in `dtype` (F16 or BF16). Writes w->codes, w->scales_dense, w->scales_sparse (PAIR) and
+ * w->tensor_scale, whose shapes/config are taken from *w. */
+SHARQ_API sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, const sharq_weight* w,
+                                   void* stream);
+
+/* Online activation preparation (SharQ page, "Core claim": adaptive N:M mask, backbone
+ * quantisation, residual against the quantised backbone, residual quantisation, fused
+ * into one operator). X: device pointer to X[M x K] row-major in `dtype` (F16 or BF16).
+ * Computes the tensor scale (NVFP4) in a first pass over X, then writes every buffer of
+ * *act, including padding rows of the tiled scale and metadata layouts. */
+SHARQ_API sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* act, void* stream);
+
+/* Y[M x N] = alpha * (sparse-FP4-GEMM(backbone, W) + dense-FP4-GEMM(residual, W)) with
+ * alpha = s_g * s_gw, accumulated in one FP32 tensor-memory accumulator and written once
+ * (SharQ page, "Core claim": a sparse FP4 GEMM for the backbone and a dense FP4 GEMM
+ * for the compensation, sharing one weight payload). Y: device pointer, row-major,
+ * y_dtype BF16 (the product) or F32. act->cfg must equal w->cfg and act->K == w->K. */
+SHARQ_API sharq_status sharq_linear(const sharq_act* act, const sharq_weight* w, void* Y,
+                          sharq_dtype y_dtype, void* stream);
+
+/* Synchronises the device, returns and clears the status word the kernels write on a
+ * bounded-wait timeout (SHARQ_OK or SHARQ_ERR_TIMEOUT), or SHARQ_ERR_CUDA if the
+ * synchronisation itself fails. */
+SHARQ_API sharq_status sharq_device_status(void);
+
+/* Static, human-readable name of a status code. */
+SHARQ_API const char* sharq_status_string(sharq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SHARQ_H */

@@ -228,16 +228,20 @@ class Prepared:
 
 
 def prepare(x: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48, residual: bool = True,
-            residual_ref: str = "quantized") -> Prepared:
+            residual_ref: str = "quantized", s_g: np.float32 | None = None) -> Prepared:
     """Online sparse-dense decomposition of one activation tensor X[M x K].
 
     residual_ref="quantized" is the method (r = x - deq(Q(backbone))); "unquantized"
-    is the ablation the page's referee asks for (r = x - backbone).
+    is the ablation the page's referee asks for (r = x - backbone). `s_g` overrides the
+    tensor scale, so that a sample of rows can be prepared exactly as inside the whole
+    tensor (rows are independent once s_g is fixed).
     """
     x = np.ascontiguousarray(x, dtype=F32)
     M, K = x.shape
     assert K % 256 == 0
-    s_g = tensor_scale(x) if fmt == NVFP4 else F32(1.0)
+    if s_g is None:
+        s_g = tensor_scale(x) if fmt == NVFP4 else F32(1.0)
+    s_g = F32(s_g)
     keep = keep_mask(x, mask)
     meta = canonical_metadata(x, mask)
     Bb = backbone_block(fmt, mask)
@@ -277,11 +281,16 @@ class QWeight:
     ws: np.ndarray  # uint8 scale codes [N, K/weight_block]
 
 
-def quantize_weight(w: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48) -> QWeight:
-    """W[K x N] -> FP4 codes stored [N x K] (K-major) with block scales along K."""
+def quantize_weight(w: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48,
+                    s_gw: np.float32 | None = None) -> QWeight:
+    """W[K x N] -> FP4 codes stored [N x K] (K-major) with block scales along K.
+
+    `s_gw` overrides the tensor scale (for quantising a sample of output columns)."""
     wt = np.ascontiguousarray(w.astype(F32).T)  # [N, K]
     N, K = wt.shape
-    s_gw = tensor_scale(wt) if fmt == NVFP4 else F32(1.0)
+    if s_gw is None:
+        s_gw = tensor_scale(wt) if fmt == NVFP4 else F32(1.0)
+    s_gw = F32(s_gw)
     Bw = weight_block(fmt, mask)
     codes, ws, _ = quant_blocks(fmt, wt.reshape(N, -1, Bw), s_gw)
     return QWeight(fmt, mask, s_gw, codes.reshape(N, K), ws.reshape(N, K // Bw))

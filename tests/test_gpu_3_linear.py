@@ -1,0 +1,144 @@
+"""GPU parity of the fused sparse + dense FP4 GEMM against the oracle's float64 product of
+the same dequantised operands.
+
+Tolerances: the oracle forms Y64 = s_g * s_gw * sum_k (B + R)[m,k] * W[n,k] exactly (every
+operand is a short dyadic number) with float64 sums. The kernel accumulates the same
+products in FP32 tensor memory, so for K <= 16384 its relative error is a few 1e-7; the
+float32 output is held to 1e-5 relative Frobenius error. The bf16 output is compared with
+bf16(Y64) rounded once from float64: the two differ only where the FP32 accumulation
+moves a value across a bf16 rounding boundary, which the 1e-3 bound (the target's) covers
+with wide margin."""
+import numpy as np
+import pytest
+
+from oracle import formats as F
+from oracle import sharq as S
+from tests.gpu_helpers import cfg_of, rel_fro, to_device, upload_act, upload_weight
+from workloads import BF16, F16, gaussian_weight, heavy_activations, tiny_activations
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-5
+TOL_BF16 = 1e-3
+
+
+def gpu_linear(act, w, out_f32=False):
+    import fp4_sparse_dense_b200 as sq
+    import torch
+    y = sq.linear(act, w, out_dtype=torch.float32 if out_f32 else torch.bfloat16)
+    torch.cuda.synchronize()
+    assert sq.sharq_device_status() == 0
+    return y.float().cpu().numpy().astype(np.float64)
+
+
+def check_y(y_gpu, y64, bf16_out):
+    if bf16_out:
+        err = rel_fro(y_gpu, F.bf16_round(y64))
+        assert err <= TOL_BF16, err
+    else:
+        err = rel_fro(y_gpu, y64)
+        assert err <= TOL_F32, err
+    return err
+
+
+GEMM_CASES = [
+    # fmt, mask, residual, M, K, N
+    ("nvfp4", "pair48", True, 128, 256, 256),
+    ("nvfp4", "pair48", True, 1, 512, 128),
+    ("nvfp4", "pair48", True, 100, 1024, 384),
+    ("nvfp4", "pair48", True, 257, 768, 512),
+    ("nvfp4", "pair48", False, 200, 512, 256),
+    ("nvfp4", "elem24", True, 130, 512, 256),
+    ("nvfp4", "elem24", False, 64, 256, 128),
+]
+MX_CASES = [
+    ("mxfp4", "pair48", True, 128, 512, 256),
+    ("mxfp4", "pair48", True, 77, 1024, 128),
+    ("mxfp4", "elem24", True, 150, 512, 256),
+    ("mxfp4", "pair48", False, 64, 256, 128),
+]
+
+
+@pytest.mark.parametrize("fmt,mask,residual,M,K,N", GEMM_CASES + MX_CASES)
+@pytest.mark.parametrize("out_f32", [True, False])
+def test_gemm_on_oracle_operands(fmt, mask, residual, M, K, N, out_f32):
+    """The GEMM alone: operands are the oracle's bytes uploaded to the GPU."""
+    rng = np.random.default_rng(M + K + N)
+    x = heavy_activations(rng, M, K)
+    w = gaussian_weight(rng, K, N)
+    p = S.prepare(x.values, fmt, mask, residual=residual)
+    qw = S.quantize_weight(w.values, fmt, mask)
+    cfg = cfg_of(fmt, mask, residual)
+    act = upload_act(S.act_buffers(p), M, K, cfg)
+    wt = upload_weight(S.weight_buffers(qw), K, N, cfg)
+    check_y(gpu_linear(act, wt, out_f32), S.linear(p, qw), not out_f32)
+
+
+@pytest.mark.parametrize("fmt,mask,residual,M,K,N", GEMM_CASES + MX_CASES)
+def test_end_to_end(fmt, mask, residual, M, K, N):
+    """prepare + quantize_weight + linear on the GPU vs the oracle chain."""
+    import fp4_sparse_dense_b200 as sq
+    rng = np.random.default_rng(3 * M + K + N)
+    x = heavy_activations(rng, M, K)
+    w = gaussian_weight(rng, K, N)
+    cfg = cfg_of(fmt, mask, residual)
+    act = sq.prepare(to_device(x), cfg)
+    wt = sq.quantize_weight(to_device(w), cfg)
+    p = S.prepare(x.values, fmt, mask, residual=residual)
+    qw = S.quantize_weight(w.values, fmt, mask)
+    check_y(gpu_linear(act, wt, True), S.linear(p, qw), False)
+
+
+def test_residual_off_is_sparse_only_product():
+    import fp4_sparse_dense_b200 as sq
+    rng = np.random.default_rng(9)
+    M, K, N = 96, 512, 256
+    x = heavy_activations(rng, M, K)
+    w = gaussian_weight(rng, K, N)
+    cfg = cfg_of("nvfp4", "pair48", False)
+    y = gpu_linear(sq.prepare(to_device(x), cfg), sq.quantize_weight(to_device(w), cfg), True)
+    p = S.prepare(x.values)
+    qw = S.quantize_weight(w.values)
+    assert rel_fro(y, S.linear_sparse_only(p, qw)) <= TOL_F32
+
+
+def test_tiny_config_end_to_end():
+    """X[16x256] fp16 with 4 outlier channels, W[256x128] fp16, element 2:4, NVFP4."""
+    import fp4_sparse_dense_b200 as sq
+    x = tiny_activations()
+    w = gaussian_weight(np.random.default_rng(1), 256, 128, F16)
+    cfg = cfg_of("nvfp4", "elem24")
+    act = sq.prepare(to_device(x), cfg)
+    wt = sq.quantize_weight(to_device(w), cfg)
+    p = S.prepare(x.values, "nvfp4", "elem24")
+    qw = S.quantize_weight(w.values, "nvfp4", "elem24")
+    y64 = S.linear(p, qw)
+    check_y(gpu_linear(act, wt, True), y64, False)
+    check_y(gpu_linear(act, wt, False), y64, True)
+
+
+@pytest.mark.parametrize("name,M,K,N,per_row", [
+    ("attn_proj", 2048, 4096, 4096, False),
+    ("mlp_gate_up", 4096, 4096, 14336, False),
+    ("mlp_down_decode", 1, 14336, 4096, True),
+    ("mlp_down_decode", 64, 14336, 4096, True),
+    ("mlp_down_prefill", 4096, 14336, 4096, True),
+])
+def test_full_size_sampled_outputs(name, M, K, N, per_row):
+    """Benchmark shapes in the benchmark's launch configuration (bf16 output): sampled
+    rows x sampled columns of Y against the oracle on those rows and columns."""
+    import fp4_sparse_dense_b200 as sq
+    rng = np.random.default_rng(M + N)
+    x = heavy_activations(rng, M, K, per_row=per_row)
+    w = gaussian_weight(rng, K, N)
+    cfg = cfg_of("nvfp4", "pair48")
+    act = sq.prepare(to_device(x), cfg)
+    wt = sq.quantize_weight(to_device(w), cfg)
+    y = gpu_linear(act, wt, False)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, min(M, 30), replace=False)]))
+    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 200, replace=False)]))
+    s_g, s_gw = S.tensor_scale(x.values), S.tensor_scale(w.values)
+    p = S.prepare(x.values[rows], s_g=s_g)
+    qw = S.quantize_weight(w.values[:, cols], s_gw=s_gw)
+    y64 = S.linear(p, qw)
+    check_y(y[np.ix_(rows, cols)], y64, True)
