@@ -121,6 +121,25 @@ class Clocks:
                 if any(r[2].replace(".", "").isdigit() for r in rows) else None}
 
 
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own token batch (independent problems, weak scaling)."""
+    return 1000 + rank
+
+
+def max_over_ranks(ms: float, dist_mod, device) -> float:
+    """Elapsed device time of the slowest rank (every rank calls this, same order)."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if dist_mod is not None and dist_mod.is_initialized() and dist_mod.get_world_size() > 1:
+        dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_step: float, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job TFLOP/s: all ranks' work divided by the slowest rank's time."""
+    return flops_per_step * world * steps / (ms_max * 1e-3) / 1e12
+
+
 def make_inputs(workload: str, seed: int):
     from workloads import gaussian_weight, heavy_activations
     M, K, N, per_row = WORKLOADS[workload]
@@ -130,14 +149,12 @@ def make_inputs(workload: str, seed: int):
     return x, w
 
 
-def cpu_baseline(workload: str, budget_s: float = 20.0, x=None, w=None):
-    """The oracle as it stands, on a bounded sample: `rows` token rows prepared and
-    multiplied by the whole (already quantised) weight. Returns (TFLOP/s, cores, sample)."""
+def cpu_baseline(workload: str, budget_s: float, x, qw):
+    """The oracle as it stands, on a bounded sample: blocks of 16 token rows prepared and
+    multiplied by the whole weight (quantised beforehand: an offline step) until the
+    budget of CPU time is used. Returns (TFLOP/s, cores, sample description)."""
     from oracle import sharq as S
     M, K, N, _ = WORKLOADS[workload]
-    if x is None:
-        x, w = make_inputs(workload, 7)
-    qw = S.quantize_weight(w.values)  # offline step, not timed
     s_g = S.tensor_scale(x.values)
     rows = 16
     t_used, n_rows = 0.0, 0
@@ -157,14 +174,16 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    from oracle import sharq as S
     M, K, N, _ = WORKLOADS[args.workload]
-    x, w = make_inputs(args.workload, 7)
+    x, w = make_inputs(args.workload, rank_seed(0))
+    qw = S.quantize_weight(w.values)  # offline step, outside the timed samples
+    budget = max(1.0, 90.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        pass  # the oracle has no state to warm
+        cpu_baseline(args.workload, budget, x, qw)
     vals = []
-    budget = max(2.0, 60.0 / max(1, args.steps))
     for _ in range(args.steps):
-        v, cores, sample = cpu_baseline(args.workload, budget, x, w)
+        v, cores, sample = cpu_baseline(args.workload, budget, x, qw)
         vals.append(v)
     value = float(np.mean(vals))
     line = {
@@ -199,7 +218,7 @@ def run_gpu(args):
     M, K, N, _ = WORKLOADS[args.workload]
     cfg = sq.Config()  # NVFP4, pair-wise 4:8, residual on
 
-    x16, w16 = make_inputs(args.workload, 1000 + rank)
+    x16, w16 = make_inputs(args.workload, rank_seed(rank))
     from tests.gpu_helpers import to_device
     n_sets = 3
     X = [to_device(x16).to(dev) for _ in range(n_sets)]
@@ -241,12 +260,9 @@ def run_gpu(args):
     ms = t_start.elapsed_time(t_end)
     prep_ms = [e[0].elapsed_time(e[1]) for e in ev]
     gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dist, dev)
     flops = 2.0 * M * N * K
-    value = flops * world * args.steps / (ms_max * 1e-3) / 1e12
+    value = job_throughput(flops, world, args.steps, ms_max)
 
     # end to end through the public API with host buffers (pinned), copies timed
     xh = [X[i].cpu().pin_memory() for i in range(n_sets)]
@@ -264,10 +280,8 @@ def run_gpu(args):
         yh.copy_(Y[i % n_sets], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = flops * world * e2e_steps / (float(te.item()) * 1e-3) / 1e12
+    e2e_value = job_throughput(flops, world, e2e_steps,
+                               max_over_ranks(e0.elapsed_time(e1), dist, dev))
     status = sq.sharq_device_status()
     assert status == 0, sq.sharq_status_string(status)
 
@@ -308,7 +322,9 @@ def run_gpu(args):
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline and world == 1:
-            v, cores, sample = cpu_baseline(args.workload, args.cpu_budget, x16, w16)
+            from oracle import sharq as S
+            qw_cpu = S.quantize_weight(w16.values)
+            v, cores, sample = cpu_baseline(args.workload, args.cpu_budget, x16, qw_cpu)
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores,
                                     "kind": "oracle", "sample": sample}
         print(json.dumps(line), flush=True)
@@ -321,8 +337,8 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
     ap.add_argument("--workload", default="mlp_gate_up", choices=list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
