@@ -155,12 +155,12 @@ def cpu_baseline(workload: str, budget_s: float, x, qw):
     budget of CPU time is used. Returns (TFLOP/s, cores, sample description)."""
     from oracle import sharq as S
     M, K, N, _ = WORKLOADS[workload]
-    s_g = S.tensor_scale(x.values)
+    amax = S.amax_of(x.values)
     rows = 16
     t_used, n_rows = 0.0, 0
     while t_used < budget_s and n_rows < M:
         t0 = time.perf_counter()
-        p = S.prepare(x.values[n_rows:n_rows + rows], s_g=s_g)
+        p = S.prepare(x.values[n_rows:n_rows + rows], amax=amax)
         S.linear(p, qw)
         t_used += time.perf_counter() - t0
         n_rows += rows

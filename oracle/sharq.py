@@ -24,9 +24,11 @@ The pages give no equations. Where they are silent the oracle takes these readin
   pairs; pairs ranked by (max |x| of the pair, then min |x| of the pair), ties to the
   lower pair index. This is the pattern the sm_100a sparse FP4 MMA accepts.
 * mask ``elem24``: in every group of 4 keep the 2 largest |x|, ties to the lower index.
-* NVFP4 tensor scale s_g = amax|X| / (6*448) in float32; block scale
-  sf = E4M3_rne_satfinite((a / 6) / s_g); d = E4M3(sf) * s_g; inv = 1 / d (one
-  correctly rounded reciprocal per block); code = E2M1_rne(x * inv) (code 0 when d == 0).
+* NVFP4 tensor constants from amax|X|, each one float32 division: the tensor scale
+  s_g = amax / (6*448) and the block-scale factor k = 448 / amax (= 1 / (6 s_g) in exact
+  arithmetic); block scale sf = E4M3_rne_satfinite(a * k) with a the block's max |x|;
+  d = E4M3(sf) * s_g; inv = 1 / d (one correctly rounded reciprocal per block);
+  code = E2M1_rne(x * inv) (code 0 when d == 0).
   Dequantised value deq = (E2M1(q) * E4M3(sf)) * s_g, all in float32 with one rounding
   per operation.
 * MXFP4 (OCP MX): e = clamp(floor(log2 a) - 2, -127, 127), scale 2^e as E8M0 code
@@ -89,17 +91,32 @@ SPARSE_VIEW_BLOCK = 32  # sparse block-scaled MMA: 4 scales per 128 logical K
 # ----------------------------------------------------------------------------- scales
 
 
+def amax_of(x: np.ndarray) -> np.float32:
+    return F32(np.max(np.abs(x.astype(F32)))) if x.size else F32(0)
+
+
+def tensor_scales(amax: np.float32) -> tuple[np.float32, np.float32]:
+    """NVFP4 per-tensor constants from amax|X| (float32, one division each):
+    s_g = amax / 2688 (the FP32 tensor scale, used to dequantise) and
+    k = 448 / amax (the block-scale factor: a / 6 / s_g in exact arithmetic)."""
+    amax = F32(amax)
+    s_g = F32(amax / GLOBAL_DIV)
+    with np.errstate(divide="ignore"):
+        k = F32(F32(448.0) / amax) if amax > 0 else F32(np.inf)
+    return s_g, k
+
+
 def tensor_scale(x: np.ndarray) -> np.float32:
     """NVFP4 FP32 tensor scale s_g = amax|X| / 2688."""
-    amax = F32(np.max(np.abs(x.astype(F32)))) if x.size else F32(0)
-    return F32(amax / GLOBAL_DIV)
+    return tensor_scales(amax_of(x))[0]
 
 
-def quant_blocks_nv(v: np.ndarray, s_g: np.float32):
+def quant_blocks_nv(v: np.ndarray, s_g: np.float32, k: np.float32):
     """NVFP4 quantisation of blocks along the last axis.
 
-    v: float32 [..., nblk, B]. Returns (codes uint8 [..., nblk, B], sf uint8 [..., nblk],
-    deq float32 [..., nblk, B]) with deq = (E2M1(q) * E4M3(sf)) * s_g in float32.
+    v: float32 [..., nblk, B]; s_g, k from tensor_scales(). Returns (codes uint8
+    [..., nblk, B], sf uint8 [..., nblk], deq float32 [..., nblk, B]) with
+    sf = E4M3(a * k), deq = (E2M1(q) * E4M3(sf)) * s_g in float32.
     """
     v = v.astype(F32)
     a = np.max(np.abs(v), axis=-1)  # float32, exact
@@ -107,7 +124,7 @@ def quant_blocks_nv(v: np.ndarray, s_g: np.float32):
         sf = np.zeros(a.shape, np.uint8)
         codes = np.zeros(v.shape, np.uint8)
         return codes, sf, np.zeros(v.shape, F32)
-    t = (a / F32(6.0)).astype(F32) / s_g  # two float32 divisions, in this order
+    t = (a * F32(k)).astype(F32)  # one float32 product per block
     sf = F.e4m3_encode_unsigned(t.astype(F32))
     sf_val = F.e4m3_decode(sf).astype(F32)  # exact
     d = (sf_val * s_g).astype(F32)
@@ -140,9 +157,10 @@ def quant_blocks_mx(v: np.ndarray):
     return codes, (e + 127).astype(np.uint8), deq
 
 
-def quant_blocks(fmt: str, v: np.ndarray, s_g: np.float32):
+def quant_blocks(fmt: str, v: np.ndarray, scales: tuple):
+    """scales = tensor_scales(amax) for NVFP4 (ignored for MXFP4)."""
     if fmt == NVFP4:
-        return quant_blocks_nv(v, s_g)
+        return quant_blocks_nv(v, *scales)
     return quant_blocks_mx(v)
 
 
@@ -228,32 +246,34 @@ class Prepared:
 
 
 def prepare(x: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48, residual: bool = True,
-            residual_ref: str = "quantized", s_g: np.float32 | None = None) -> Prepared:
+            residual_ref: str = "quantized", amax: np.float32 | None = None) -> Prepared:
     """Online sparse-dense decomposition of one activation tensor X[M x K].
 
     residual_ref="quantized" is the method (r = x - deq(Q(backbone))); "unquantized"
-    is the ablation the page's referee asks for (r = x - backbone). `s_g` overrides the
-    tensor scale, so that a sample of rows can be prepared exactly as inside the whole
-    tensor (rows are independent once s_g is fixed).
+    is the ablation the page's referee asks for (r = x - backbone). `amax` overrides the
+    tensor's max |x|, so that a sample of rows can be prepared exactly as inside the
+    whole tensor (rows are independent once the tensor constants are fixed).
     """
     x = np.ascontiguousarray(x, dtype=F32)
     M, K = x.shape
     assert K % 256 == 0
-    if s_g is None:
-        s_g = tensor_scale(x) if fmt == NVFP4 else F32(1.0)
-    s_g = F32(s_g)
+    if fmt == NVFP4:
+        sc = tensor_scales(amax_of(x) if amax is None else amax)
+    else:
+        sc = (F32(1.0), F32(1.0))
+    s_g = sc[0]
     keep = keep_mask(x, mask)
     meta = canonical_metadata(x, mask)
     Bb = backbone_block(fmt, mask)
     if mask == PAIR48:
         comp = x[keep].reshape(M, K // 2)  # kept values in K order (row-major boolean gather)
-        codes, bs, deq_c = quant_blocks(fmt, comp.reshape(M, -1, 16), s_g)
+        codes, bs, deq_c = quant_blocks(fmt, comp.reshape(M, -1, 16), sc)
         bq = codes.reshape(M, K // 2)
         b_deq = np.zeros((M, K), F32)
         b_deq[keep] = deq_c.reshape(-1)
     else:
         b = np.where(keep, x, F32(0))
-        codes, bs, deq = quant_blocks(fmt, b.reshape(M, -1, Bb), s_g)
+        codes, bs, deq = quant_blocks(fmt, b.reshape(M, -1, Bb), sc)
         bq = codes.reshape(M, K)
         b_deq = np.where(keep, deq.reshape(M, K), F32(0)).astype(F32)
     bs = bs.reshape(M, K // Bb)
@@ -262,7 +282,7 @@ def prepare(x: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48, residual: bool 
         sub = b_deq if residual_ref == "quantized" else np.where(keep, x, F32(0))
         r = np.where(keep, (x - sub).astype(F32), x).astype(F32)
         Br = residual_block(fmt)
-        rc, rsc, rd = quant_blocks(fmt, r.reshape(M, -1, Br), s_g)
+        rc, rsc, rd = quant_blocks(fmt, r.reshape(M, -1, Br), sc)
         rq = rc.reshape(M, K)
         rs = rsc.reshape(M, K // Br)
         r_deq = rd.reshape(M, K)
@@ -282,17 +302,19 @@ class QWeight:
 
 
 def quantize_weight(w: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48,
-                    s_gw: np.float32 | None = None) -> QWeight:
+                    amax: np.float32 | None = None) -> QWeight:
     """W[K x N] -> FP4 codes stored [N x K] (K-major) with block scales along K.
 
-    `s_gw` overrides the tensor scale (for quantising a sample of output columns)."""
+    `amax` overrides max |W| (for quantising a sample of output columns)."""
     wt = np.ascontiguousarray(w.astype(F32).T)  # [N, K]
     N, K = wt.shape
-    if s_gw is None:
-        s_gw = tensor_scale(wt) if fmt == NVFP4 else F32(1.0)
-    s_gw = F32(s_gw)
+    if fmt == NVFP4:
+        sc = tensor_scales(amax_of(wt) if amax is None else amax)
+    else:
+        sc = (F32(1.0), F32(1.0))
+    s_gw = sc[0]
     Bw = weight_block(fmt, mask)
-    codes, ws, _ = quant_blocks(fmt, wt.reshape(N, -1, Bw), s_gw)
+    codes, ws, _ = quant_blocks(fmt, wt.reshape(N, -1, Bw), sc)
     return QWeight(fmt, mask, s_gw, codes.reshape(N, K), ws.reshape(N, K // Bw))
 
 

@@ -91,11 +91,11 @@ def test_prep_full_size_sampled_rows(name, M, K, per_row):
     x = heavy_activations(rng, M, K, per_row=per_row)
     act = run_prep(x, "nvfp4", "pair48")
     got = act_bytes(act)
-    s_g = S.tensor_scale(x.values)
-    assert got["tensor_scale"][0] == s_g
+    amax = S.amax_of(x.values)
+    assert got["tensor_scale"][0] == S.tensor_scales(amax)[0]
     rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 46, replace=False)]))
     g = sampled_act_rows(got, rows, M, K, "nvfp4", "pair48")
-    p = S.prepare(x.values[rows], "nvfp4", "pair48", s_g=s_g)
+    p = S.prepare(x.values[rows], "nvfp4", "pair48", amax=amax)
     from oracle import layouts as L
     assert np.array_equal(g["bq"], L.pack_nibbles(p.bq))
     assert np.array_equal(g["bs"], p.bs)

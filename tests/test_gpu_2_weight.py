@@ -36,10 +36,10 @@ def test_weight_quant_full_size_sampled_columns():
     rng = np.random.default_rng(5)
     w = gaussian_weight(rng, K, N)
     got = weight_bytes(run_wq(w, "nvfp4", "pair48"))
-    s_gw = S.tensor_scale(w.values)
-    assert got["tensor_scale"][0] == s_gw
+    amax = S.amax_of(w.values)
+    assert got["tensor_scale"][0] == S.tensor_scales(amax)[0]
     cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 62, replace=False)]))
-    q = S.quantize_weight(w.values[:, cols], "nvfp4", "pair48", s_gw=s_gw)
+    q = S.quantize_weight(w.values[:, cols], "nvfp4", "pair48", amax=amax)
     codes = got["codes"].reshape(N, K // 2)[cols]
     assert np.array_equal(codes, L.pack_nibbles(q.wq))
     assert np.array_equal(L.from_scale_layout(got["scales_sparse"], N, K // 32)[cols], q.ws)

@@ -137,8 +137,7 @@ def test_full_size_sampled_outputs(name, M, K, N, per_row):
     y = gpu_linear(act, wt, False)
     rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, min(M, 30), replace=False)]))
     cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 200, replace=False)]))
-    s_g, s_gw = S.tensor_scale(x.values), S.tensor_scale(w.values)
-    p = S.prepare(x.values[rows], s_g=s_g)
-    qw = S.quantize_weight(w.values[:, cols], s_gw=s_gw)
+    p = S.prepare(x.values[rows], amax=S.amax_of(x.values))
+    qw = S.quantize_weight(w.values[:, cols], amax=S.amax_of(w.values))
     y64 = S.linear(p, qw)
     check_y(y[np.ix_(rows, cols)], y64, True)

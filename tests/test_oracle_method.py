@@ -138,12 +138,14 @@ def test_backbone_plus_residual_is_exact(fmt, mask):
 def test_nvfp4_scale_and_codes_are_nearest():
     rng = np.random.default_rng(4)
     x = heavy_activations(rng, 16, 1024).values
-    s_g = S.tensor_scale(x)
+    s_g, k = S.tensor_scales(np.abs(x).max())
     v = x.reshape(16, -1, 16)
-    codes, sf, deq = S.quant_blocks_nv(v, s_g)
+    codes, sf, deq = S.quant_blocks_nv(v, s_g, k)
     a = np.abs(v).max(-1)
     # the scale argument is formed in float32 (the precision the recipe fixes)
-    t = ((a / np.float32(6)).astype(np.float32) / s_g).astype(np.float32).astype(np.float64)
+    t = (a * k).astype(np.float32).astype(np.float64)
+    # k is 1 / (6 s_g) up to the two float32 roundings
+    assert abs(float(k) * 6 * float(s_g) - 1) < 2.5e-7
     # sf is the nearest E4M3 value to t (saturating at 448), by brute force over the table
     best = np.abs(np.minimum(t, 448)[..., None] - F.E4M3_TABLE).min(-1)
     assert np.array_equal(np.abs(np.minimum(t, 448) - F.e4m3_decode(sf)), best)
@@ -189,7 +191,7 @@ def test_residual_recovers_error_on_outlier_inputs(fmt):
     p = S.prepare(x, fmt, S.PAIR48)
     err = np.linalg.norm(p.b_deq + p.r_deq - x)
     _, _, plain = S.quant_blocks(fmt, x.reshape(128, -1, S.residual_block(fmt)),
-                                 S.tensor_scale(x) if fmt == S.NVFP4 else np.float32(1))
+                                 S.tensor_scales(np.abs(x).max()))
     err_plain = np.linalg.norm(plain.reshape(x.shape) - x)
     pu = S.prepare(x, fmt, S.PAIR48, residual_ref="unquantized")
     err_unq = np.linalg.norm(pu.b_deq + pu.r_deq - x)
