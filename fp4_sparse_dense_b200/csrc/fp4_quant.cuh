@@ -1,25 +1,28 @@
 // Block quantisation recipes shared by the activation and weight kernels (device code).
 //
-// NVFP4: sf = E4M3_rne((a / 6) / s_g) with a the block's max |v|; d = E4M3(sf) * s_g;
-// inv = 1 / d (one correctly rounded reciprocal per block); q = E2M1_rne(v * inv).
+// NVFP4: sf = E4M3_rne(a * k) with a the block's max |v| and k = 448 / amax per tensor;
+// d = E4M3(sf) * s_g with s_g = amax / 2688; inv = 1 / d (one correctly rounded
+// reciprocal per block); q = E2M1_rne(v * inv).
 // MXFP4 (OCP MX): e = clamp(floor(log2 a) - 2, -127, 127); q = E2M1_rne(v * 2^-e).
 // Every float operation is an explicit round-to-nearest intrinsic so that the compiler
 // cannot contract or reassociate them.
 #pragma once
 #include <cstdint>
+#include <cuda_fp16.h>
 
 #include "fp4_device.cuh"
 #include "sharq_internal.h"
 
 namespace sharq {
 
-// NVFP4 quantisation of N values with one E4M3 block scale:
-//   sf = E4M3((a / 6) / s_g), d = E4M3(sf) * s_g, inv = 1 / d, q = E2M1(v * inv).
+// NVFP4 quantisation of N values with one E4M3 block scale, given the tensor constants
+// s_g = amax / 2688 and k = 448 / amax:
+//   sf = E4M3(a * k), d = E4M3(sf) * s_g, inv = 1 / d, q = E2M1(v * inv).
 // Returns the scale code; codes (4 bits each, v[0] lowest) go to `packed`; deq[i] =
-// (E2M1(q_i) * E4M3(sf)) * s_g when want_deq.
+// (E2M1(q_i) * E4M3(sf)) * s_g when WANT_DEQ.
 template <int N, bool WANT_DEQ>
-__device__ __forceinline__ uint32_t quant_nv(const float* v, float s_g, uint32_t* packed,
-                                             float* deq) {
+__device__ __forceinline__ uint32_t quant_nv(const float* v, float s_g, float k,
+                                             uint32_t* packed, float* deq) {
   float a = 0.f;
 #pragma unroll
   for (int i = 0; i < N; ++i) a = fmaxf(a, fabsf(v[i]));
@@ -27,26 +30,38 @@ __device__ __forceinline__ uint32_t quant_nv(const float* v, float s_g, uint32_t
   float sf_val = 0.f, inv = 0.f;
   bool live = false;
   if (s_g > 0.f) {
-    sf = cvt_e4m3(__fdiv_rn(__fdiv_rn(a, 6.0f), s_g));
+    sf = cvt_e4m3(__fmul_rn(a, k));
     sf_val = e4m3_value(sf);
     const float d = __fmul_rn(sf_val, s_g);
     live = d > 0.f;
     inv = live ? __frcp_rn(d) : 0.f;
   }
+  const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
   for (int w = 0; w < N / 8; ++w) {
     const float* s = v + 8 * w;
-    packed[w] = live ? cvt_e2m1x8(__fmul_rn(s[0], inv), __fmul_rn(s[1], inv),
-                                  __fmul_rn(s[2], inv), __fmul_rn(s[3], inv),
-                                  __fmul_rn(s[4], inv), __fmul_rn(s[5], inv),
-                                  __fmul_rn(s[6], inv), __fmul_rn(s[7], inv))
-                     : 0u;
+    const float2 p0 = mul2_rn(make_float2(s[0], s[1]), inv2);
+    const float2 p1 = mul2_rn(make_float2(s[2], s[3]), inv2);
+    const float2 p2 = mul2_rn(make_float2(s[4], s[5]), inv2);
+    const float2 p3 = mul2_rn(make_float2(s[6], s[7]), inv2);
+    packed[w] = live ? cvt_e2m1x8(p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y) : 0u;
   }
   if (WANT_DEQ) {
+    // E2M1(q) * E4M3(sf) is exact in f16 (at most 6 significant bits, magnitude in
+    // [2^-10, 2688]); one float32 rounding for the tensor scale.
+    const __half2 sf2 = __float2half2_rn(sf_val);
+    const float2 sg2 = make_float2(s_g, s_g);
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-      const uint32_t c = (packed[i / 8] >> (4 * (i % 8))) & 0xFu;
-      deq[i] = __fmul_rn(__fmul_rn(e2m1_value(c), sf_val), s_g);
+    for (int w = 0; w < N / 8; ++w) {
+      uint32_t h[4];
+      e2m1x8_to_f16x2(packed[w], h);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f =
+            mul2_rn(__half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[j]), sf2)), sg2);
+        deq[8 * w + 2 * j] = f.x;
+        deq[8 * w + 2 * j + 1] = f.y;
+      }
     }
   }
   return sf;
@@ -66,30 +81,49 @@ __device__ __forceinline__ uint32_t quant_mx(const float* v, uint32_t* packed, f
   const bool live = a > 0.f;
   if (!live) e = -127;
   const float scale = __uint_as_float(uint32_t(127 - e) << 23);  // 2^-e, -e in [-125, 127]
+  const float2 sc2 = make_float2(scale, scale);
 #pragma unroll
   for (int w = 0; w < N / 8; ++w) {
     const float* s = v + 8 * w;
-    packed[w] = live ? cvt_e2m1x8(__fmul_rn(s[0], scale), __fmul_rn(s[1], scale),
-                                  __fmul_rn(s[2], scale), __fmul_rn(s[3], scale),
-                                  __fmul_rn(s[4], scale), __fmul_rn(s[5], scale),
-                                  __fmul_rn(s[6], scale), __fmul_rn(s[7], scale))
-                     : 0u;
+    const float2 p0 = mul2_rn(make_float2(s[0], s[1]), sc2);
+    const float2 p1 = mul2_rn(make_float2(s[2], s[3]), sc2);
+    const float2 p2 = mul2_rn(make_float2(s[4], s[5]), sc2);
+    const float2 p3 = mul2_rn(make_float2(s[6], s[7]), sc2);
+    packed[w] = live ? cvt_e2m1x8(p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y) : 0u;
   }
   if (WANT_DEQ) {
     const float p2 = pow2f(e);
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-      const uint32_t c = (packed[i / 8] >> (4 * (i % 8))) & 0xFu;
-      deq[i] = __fmul_rn(e2m1_value(c), p2);
+    for (int w = 0; w < N / 8; ++w) {
+      uint32_t h[4];
+      e2m1x8_to_f16x2(packed[w], h);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[j]));
+        deq[8 * w + 2 * j] = __fmul_rn(f.x, p2);
+        deq[8 * w + 2 * j + 1] = __fmul_rn(f.y, p2);
+      }
     }
   }
   return uint32_t(e + 127);
 }
 
+// Per-tensor constants of the NVFP4 recipe from amax (one float32 division each).
+struct TensorConsts {
+  float s_g;  // amax / 2688: the FP32 tensor scale
+  float k;    // 448 / amax: block-scale factor
+};
+__device__ __forceinline__ TensorConsts tensor_consts(float amax) {
+  TensorConsts c;
+  c.s_g = __fdiv_rn(amax, 2688.0f);
+  c.k = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+  return c;
+}
+
 template <int FMT, int N, bool WANT_DEQ>
-__device__ __forceinline__ uint32_t quant_block(const float* v, float s_g, uint32_t* packed,
+__device__ __forceinline__ uint32_t quant_block(const float* v, TensorConsts c, uint32_t* packed,
                                                 float* deq) {
-  if (FMT == SHARQ_NVFP4) return quant_nv<N, WANT_DEQ>(v, s_g, packed, deq);
+  if (FMT == SHARQ_NVFP4) return quant_nv<N, WANT_DEQ>(v, c.s_g, c.k, packed, deq);
   return quant_mx<N, WANT_DEQ>(v, packed, deq);
 }
 

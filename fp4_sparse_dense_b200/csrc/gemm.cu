@@ -9,17 +9,18 @@
 // block-scaled MMAs (residual, 64 K each), all accumulating into one FP32 accumulator in
 // tensor memory, which one epilogue scales by alpha = s_g * s_gw and writes once.
 //
-// CTA organisation (persistent, one CTA per SM, 6 warps):
+// CTA organisation (persistent, one CTA per SM, 10 warps):
 //   warp 0      TMA producer: FP4 tiles by tensor-map loads, scales and metadata by
 //               1-D bulk copies, all completing on the stage's "full" mbarrier;
 //   warp 1      tensor-memory owner and single-thread MMA issuer: copies the stage's
 //               scales / metadata into tensor memory (tcgen05.cp) and issues the MMAs;
 //               tcgen05.commit releases the stage and, after the last K step, the
 //               accumulator;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows, scale, convert, store.
-// Tensor memory: columns [0, BN) accumulator, columns from 256 the scale factors and the
-// sparse metadata of the current K step (single-buffered: the copy and the MMAs are
-// issued by one thread and execute in issue order).
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator into registers, release of the
+//               accumulator, then scale, convert and store (overlapping the next tile).
+// Tensor memory: columns [0, BN) accumulator; from column 256 two buffers of the scale
+// factors and sparse metadata, used by alternate K steps, so that the copies of step k+1
+// never write columns the MMAs of step k may still read.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -30,6 +31,8 @@
 namespace sharq {
 
 constexpr int kMaxSmem = 232448;  // 227 KB opt-in dynamic shared memory per CTA
+constexpr int kEpiThreads = 256;  // 8 epilogue warps
+constexpr int kThreads = 64 + kEpiThreads;
 
 template <int FMT, bool PAIR, bool RES, int BN>
 struct GemmCfg {
@@ -67,7 +70,9 @@ struct GemmCfg {
   static constexpr int COL_SWS = COL_SWD + (DENSE_W ? DCH * (BN / 32) : 0);
   static constexpr int COL_E = COL_SWS + (PAIR ? 2 * (BN / 32) : 0);
   static constexpr int COL_END = COL_E + (PAIR ? 4 : 0);
-  static_assert(COL_END <= 512, "tensor memory overflow");
+  // scales / metadata are double-buffered: K step kt uses columns + (kt & 1) * SF_SPAN
+  static constexpr int SF_SPAN = (COL_END - COL_SFR + 3) / 4 * 4;
+  static_assert(COL_SFR + 2 * SF_SPAN <= 512, "tensor memory overflow");
   static_assert(STAGES >= 2, "not enough shared memory for two stages");
   // instruction descriptors (block-scaled kinds): E2M1 A and B, M = 128, N = BN
   static constexpr uint32_t IDESC_BASE =
@@ -76,7 +81,7 @@ struct GemmCfg {
 };
 
 template <int FMT, bool PAIR, bool RES, int BN, bool OUT_F32>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     sharq_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_r, const GemmParams p) {
@@ -104,7 +109,7 @@ __global__ void __launch_bounds__(192, 1)
       ptx::mbar_init(ptx::smem_u32(empty_bar + s), 1);
     }
     ptx::mbar_init(ptx::smem_u32(tfull_bar), 1);
-    ptx::mbar_init(ptx::smem_u32(tempty_bar), 128);
+    ptx::mbar_init(ptx::smem_u32(tempty_bar), kEpiThreads);
     ptx::mbar_init(ptx::smem_u32(drain_bar), 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -200,32 +205,34 @@ __global__ void __launch_bounds__(192, 1)
           }
           ptx::tc_fence_after();
           const uint32_t st = ptx::smem_u32(smem + s * C::STAGE);
+          // this K step's half of the double-buffered scale / metadata columns
+          const uint32_t tb = tbase + uint32_t(kt & 1) * C::SF_SPAN;
           // ---- scale factors and metadata of this K step into tensor memory
           if (PAIR) {
-            ptx::tmem_cp_128x128b(tbase + C::COL_E, ptx::smem_desc(st + C::OFF_E, 16, 128, 0));
+            ptx::tmem_cp_128x128b(tb + C::COL_E, ptx::smem_desc(st + C::OFF_E, 16, 128, 0));
             for (int j = 0; j < 2; ++j) {
-              ptx::tmem_cp_32x128b_x4(tbase + C::COL_SFB + 4 * j,
+              ptx::tmem_cp_32x128b_x4(tb + C::COL_SFB + 4 * j,
                                       ptx::smem_desc(st + C::OFF_SFB + 512 * j, 16, 128, 0));
               for (int rb = 0; rb < BN / 128; ++rb)
                 ptx::tmem_cp_32x128b_x4(
-                    tbase + C::COL_SWS + j * (BN / 32) + 4 * rb,
+                    tb + C::COL_SWS + j * (BN / 32) + 4 * rb,
                     ptx::smem_desc(st + C::OFF_SWS + (rb * 2 + j) * 512, 16, 128, 0));
             }
           } else {
             for (int c = 0; c < C::DCH; ++c)
-              ptx::tmem_cp_32x128b_x4(tbase + C::COL_SFB + 4 * c,
+              ptx::tmem_cp_32x128b_x4(tb + C::COL_SFB + 4 * c,
                                       ptx::smem_desc(st + C::OFF_SFB + 512 * c, 16, 128, 0));
           }
           if (RES) {
             for (int c = 0; c < C::DCH; ++c)
-              ptx::tmem_cp_32x128b_x4(tbase + C::COL_SFR + 4 * c,
+              ptx::tmem_cp_32x128b_x4(tb + C::COL_SFR + 4 * c,
                                       ptx::smem_desc(st + C::OFF_SFR + 512 * c, 16, 128, 0));
           }
           if (C::DENSE_W) {
             for (int c = 0; c < C::DCH; ++c)
               for (int rb = 0; rb < BN / 128; ++rb)
                 ptx::tmem_cp_32x128b_x4(
-                    tbase + C::COL_SWD + c * (BN / 32) + 4 * rb,
+                    tb + C::COL_SWD + c * (BN / 32) + 4 * rb,
                     ptx::smem_desc(st + C::OFF_SWD + (rb * C::DCH + c) * 512, 16, 128, 0));
           }
           // ---- MMAs: backbone then residual, one accumulator
@@ -234,8 +241,8 @@ __global__ void __launch_bounds__(192, 1)
             for (int j = 0; j < 2; ++j) {
               const uint64_t a = ptx::smem_desc(st + C::OFF_B + 32 * j, 16, 512, 4);
               const uint64_t b = ptx::smem_desc(st + C::OFF_W + 64 * j, 16, 1024, 2);
-              ptx::mma_sp_nvf4(tbase, a, b, tbase + C::COL_E + 2 * j, idesc_s,
-                               tbase + C::COL_SFB + 4 * j, tbase + C::COL_SWS + j * (BN / 32), acc);
+              ptx::mma_sp_nvf4(tbase, a, b, tb + C::COL_E + 2 * j, idesc_s,
+                               tb + C::COL_SFB + 4 * j, tb + C::COL_SWS + j * (BN / 32), acc);
               acc = 1u;
             }
           } else {
@@ -243,13 +250,13 @@ __global__ void __launch_bounds__(192, 1)
               const uint64_t a = ptx::smem_desc(st + C::OFF_B + 32 * i, 16, 1024, 2);
               const uint64_t b = ptx::smem_desc(st + C::OFF_W + 32 * i, 16, 1024, 2);
               if (C::NV) {
-                ptx::mma_nvf4(tbase, a, b, idesc_d, tbase + C::COL_SFB + 4 * i,
-                              tbase + C::COL_SWD + i * (BN / 32), acc);
+                ptx::mma_nvf4(tbase, a, b, idesc_d, tb + C::COL_SFB + 4 * i,
+                              tb + C::COL_SWD + i * (BN / 32), acc);
               } else {
                 const uint32_t id = 2u * uint32_t(i & 1);
                 ptx::mma_mxf4(tbase, a, b, idesc_d | (id << 29) | (id << 4),
-                              (tbase + C::COL_SFB + 4 * (i >> 1)) | (id << 30),
-                              (tbase + C::COL_SWD + (i >> 1) * (BN / 32)) | (id << 30), acc);
+                              (tb + C::COL_SFB + 4 * (i >> 1)) | (id << 30),
+                              (tb + C::COL_SWD + (i >> 1) * (BN / 32)) | (id << 30), acc);
               }
               acc = 1u;
             }
@@ -259,13 +266,13 @@ __global__ void __launch_bounds__(192, 1)
               const uint64_t a = ptx::smem_desc(st + C::OFF_R + 32 * i, 16, 1024, 2);
               const uint64_t b = ptx::smem_desc(st + C::OFF_W + 32 * i, 16, 1024, 2);
               if (C::NV) {
-                ptx::mma_nvf4(tbase, a, b, idesc_d, tbase + C::COL_SFR + 4 * i,
-                              tbase + C::COL_SWD + i * (BN / 32), 1u);
+                ptx::mma_nvf4(tbase, a, b, idesc_d, tb + C::COL_SFR + 4 * i,
+                              tb + C::COL_SWD + i * (BN / 32), 1u);
               } else {
                 const uint32_t id = 2u * uint32_t(i & 1);
                 ptx::mma_mxf4(tbase, a, b, idesc_d | (id << 29) | (id << 4),
-                              (tbase + C::COL_SFR + 4 * (i >> 1)) | (id << 30),
-                              (tbase + C::COL_SWD + (i >> 1) * (BN / 32)) | (id << 30), 1u);
+                              (tb + C::COL_SFR + 4 * (i >> 1)) | (id << 30),
+                              (tb + C::COL_SWD + (i >> 1) * (BN / 32)) | (id << 30), 1u);
               }
             }
           }
@@ -282,7 +289,13 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // tensor-memory lane quarter this warp may access
+    // Eight warps: warp w reads tensor-memory lane quarter w % 4 (rows) and column half
+    // (w - 2) / 4. Each thread pulls its row's BN/2 accumulator columns into registers,
+    // releases the accumulator (so the next tile's MMAs start at once), then scales,
+    // converts and stores while the tensor cores run ahead.
+    constexpr int HALF = BN / 2;
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const float alpha = __fmul_rn(p.act_ts[0], p.w_ts[0]);
     int tcount = 0;
     bool ok = true;
@@ -294,41 +307,39 @@ __global__ void __launch_bounds__(192, 1)
       }
       ptx::tc_fence_after();
       const int row = mb * 128 + quarter * 32 + lane;
-      const uint32_t taddr = tbase + (uint32_t(quarter * 32) << 16);
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
-        ptx::tmem_ld_wait();
-        if (row < p.M) {
-          const size_t off = size_t(row) * p.N + size_t(nb) * BN + c * 32;
-          if (OUT_F32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + off);
+      const uint32_t taddr = tbase + (uint32_t(quarter * 32) << 16) + uint32_t(half * HALF);
+      uint32_t v[HALF];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__fmul_rn(__uint_as_float(v[4 * i]), alpha),
-                                   __fmul_rn(__uint_as_float(v[4 * i + 1]), alpha),
-                                   __fmul_rn(__uint_as_float(v[4 * i + 2]), alpha),
-                                   __fmul_rn(__uint_as_float(v[4 * i + 3]), alpha));
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + off);
+      for (int c = 0; c < HALF / 32; ++c) ptx::tmem_ld_32x32b_x32(taddr + c * 32, v + 32 * c);
+      ptx::tmem_ld_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_u32(tempty_bar));
+      if (row < p.M) {
+        const size_t off = size_t(row) * p.N + size_t(nb) * BN + size_t(half) * HALF;
+        if (OUT_F32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + off);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint32_t w4[4];
+          for (int i = 0; i < HALF / 4; ++i)
+            dst[i] = make_float4(__fmul_rn(__uint_as_float(v[4 * i]), alpha),
+                                 __fmul_rn(__uint_as_float(v[4 * i + 1]), alpha),
+                                 __fmul_rn(__uint_as_float(v[4 * i + 2]), alpha),
+                                 __fmul_rn(__uint_as_float(v[4 * i + 3]), alpha));
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + off);
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const __nv_bfloat162 b2 =
-                    __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[8 * i + 2 * h]), alpha),
-                                          __fmul_rn(__uint_as_float(v[8 * i + 2 * h + 1]), alpha));
-                w4[h] = *reinterpret_cast<const uint32_t*>(&b2);
-              }
-              dst[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int i = 0; i < HALF / 8; ++i) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_bfloat162 b2 =
+                  __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[8 * i + 2 * h]), alpha),
+                                        __fmul_rn(__uint_as_float(v[8 * i + 2 * h + 1]), alpha));
+              w4[h] = *reinterpret_cast<const uint32_t*>(&b2);
             }
+            dst[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
       }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(ptx::smem_u32(tempty_bar));
     }
     if (!ok && lane == 0) atomicExch(p.status, unsigned(SHARQ_ERR_TIMEOUT));
   }
@@ -349,7 +360,7 @@ static cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, int num_sms,
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  kern<<<grid, 192, C::SMEM, st>>>(m.w, m.b, m.r, p);
+  kern<<<grid, kThreads, C::SMEM, st>>>(m.w, m.b, m.r, p);
   return cudaGetLastError();
 }
 

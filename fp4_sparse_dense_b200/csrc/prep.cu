@@ -30,13 +30,20 @@ template <bool BF16>
 __global__ void __launch_bounds__(512) amax_kernel(const uint4* __restrict__ X, size_t n16,
                                                   unsigned int* amax_bits) {
   uint32_t m = 0;  // two packed 15-bit magnitudes
-  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n16;
-       i += size_t(gridDim.x) * blockDim.x) {
-    const uint4 v = __ldg(X + i);
-    m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
-    m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
-    m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
-    m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+  const size_t stride = size_t(gridDim.x) * blockDim.x;
+  // four independent 16-byte loads in flight per thread
+  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n16; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      v[j] = i + j * stride < n16 ? __ldg(X + i + j * stride) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      m = __vmaxu2(m, v[j].x & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v[j].y & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v[j].z & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v[j].w & 0x7FFF7FFFu);
+    }
   }
   uint32_t h = max(m & 0xFFFFu, m >> 16);
   for (int off = 16; off; off >>= 1) h = max(h, __shfl_xor_sync(0xFFFFFFFFu, h, off));
@@ -50,10 +57,221 @@ __global__ void __launch_bounds__(512) amax_kernel(const uint4* __restrict__ X, 
   }
 }
 
-// ------------------------------------------------------------------------------ prep
+// ------------------------------------------------------------------------------ pair 4:8
 
-template <bool BF16, int FMT, int MASK, bool RESIDUAL>
-__global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
+// Entry of the top-2-of-4 decision table. Bit b of `idx` is one comparison "candidate i
+// beats candidate j" (i < j; a tie is won by i) in the order (0,1) (0,2) (0,3) (1,2)
+// (1,3) (2,3). A candidate is kept when fewer than two others beat it; the entry is the
+// metadata nibble i0 | i1 << 2 of the two kept candidates (i0 < i1).
+__device__ __forceinline__ uint8_t top2_entry(int idx) {
+  const int c01 = idx & 1, c02 = (idx >> 1) & 1, c03 = (idx >> 2) & 1;
+  const int c12 = (idx >> 3) & 1, c13 = (idx >> 4) & 1, c23 = (idx >> 5) & 1;
+  const int rank[4] = {3 - c01 - c02 - c03, c01 + 2 - c12 - c13, c02 + c12 + 1 - c23,
+                       c03 + c13 + c23};
+  int i0 = -1, i1 = -1;
+  for (int j = 0; j < 4; ++j)
+    if (rank[j] < 2) {
+      if (i0 < 0) i0 = j;
+      else if (i1 < 0) i1 = j;
+    }
+  if (i0 < 0 || i1 < 0) return 0x4;  // not reachable from a total order
+  return uint8_t(i0 | (i1 << 2));
+}
+
+// Ranking key of a pair (two 16-bit inputs in one word): the larger 15-bit magnitude in
+// the high half, the smaller in the low half. For bf16 and fp16 the magnitude order of
+// the values is the unsigned order of these bit fields.
+__device__ __forceinline__ uint32_t pair_key(uint32_t w) {
+  const uint32_t m = w & 0x7FFF7FFFu;
+  const uint32_t sw = __byte_perm(m, 0, 0x1032);
+  return __byte_perm(__vmaxu2(m, sw), __vminu2(m, sw), 0x3254);
+}
+
+template <bool BF16>
+__device__ __forceinline__ float lo16(uint32_t w) { return in_to_float<BF16>(w & 0xFFFFu); }
+template <bool BF16>
+__device__ __forceinline__ float hi16(uint32_t w) { return in_to_float<BF16>(w >> 16); }
+
+// Pair-wise 4:8 mask: in every 8 consecutive K keep the 2 of the 4 adjacent pairs with the
+// largest (max |x|, min |x|), ties to the lower pair; the kept values (compressed, 16 per
+// 32 K) form one backbone block; the residual is taken against their dequantised values.
+//
+// Persistent and warp-independent: a warp item is 4 rows x 256 K (lane = row * 8 + unit,
+// unit = 32 K); warps walk the items with a grid stride, loading the next item while
+// computing the current one. Scale and metadata bytes of neighbouring lanes are gathered
+// with shuffles into 32-bit stores, so no CTA barrier is needed inside the loop.
+template <bool BF16, int FMT, bool RESIDUAL>
+__global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
+  constexpr int RB = FMT == SHARQ_NVFP4 ? 16 : 32;  // residual block
+  __shared__ uint8_t s_top2[64];
+  if (threadIdx.x < 64) s_top2[threadIdx.x] = top2_entry(threadIdx.x);
+
+  TensorConsts tc{1.f, 1.f};
+  if (FMT == SHARQ_NVFP4) {
+    tc = tensor_consts(__uint_as_float(*reinterpret_cast<const unsigned int*>(p.amax)));
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.tensor_scale = tc.s_g;
+  } else if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *p.tensor_scale = 1.0f;
+  }
+  __syncthreads();  // decision table ready
+
+  const int K = p.K, M = p.M, Mp = p.Mp;
+  const int KS = K / 256;                   // 256-K slices
+  const int n_items = (Mp / 4) * KS;
+  const int lane = threadIdx.x & 31;
+  const int u = lane & 7;                   // 32-K unit inside the slice
+  const int rsub = lane >> 3;               // row inside the item
+  const int stride = gridDim.x * (blockDim.x >> 5);
+  const uint16_t* X = static_cast<const uint16_t*>(p.X);
+  const size_t scols_b = size_t(K) / 32 / 4;  // 512-byte chunks per 128 rows (backbone)
+  const size_t scols_r = size_t(K) / RB / 4;  // (residual)
+
+  int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  uint4 cur[4];
+  auto load = [&](int it, uint4* dst) {
+    const int row = (it / KS) * 4 + rsub;
+    if (it < n_items && row < M) {
+      const uint4* src =
+          reinterpret_cast<const uint4*>(X + size_t(row) * K + size_t(it % KS) * 256 + u * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = __ldg(src + i);
+    }
+  };
+  load(item, cur);
+
+#pragma unroll 1
+  for (; item < n_items; item += stride) {
+    uint4 nxt[4];
+    load(item + stride, nxt);
+    const int q = item % KS;
+    const int row = (item / KS) * 4 + rsub;
+    const int k0 = q * 256 + u * 32;
+    const bool live = row < M;
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      w[4 * i + 0] = cur[i].x; w[4 * i + 1] = cur[i].y;
+      w[4 * i + 2] = cur[i].z; w[4 * i + 3] = cur[i].w;
+    }
+
+    uint32_t meta = 0x4444u, bsf = 0, rsf0 = 0, rsf1 = 0;
+    if (live) {
+      // ---- mask: one table lookup per group of 4 pairs
+      int sel0[4], sel1[4];
+      float comp[16];
+      meta = 0;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const uint32_t ka = pair_key(w[4 * g]), kb = pair_key(w[4 * g + 1]);
+        const uint32_t kc = pair_key(w[4 * g + 2]), kd = pair_key(w[4 * g + 3]);
+        const int idx = int(ka >= kb) | (int(ka >= kc) << 1) | (int(ka >= kd) << 2) |
+                        (int(kb >= kc) << 3) | (int(kb >= kd) << 4) | (int(kc >= kd) << 5);
+        const uint32_t nib = s_top2[idx];
+        const int i0 = int(nib & 3u), i1 = int(nib >> 2);
+        sel0[g] = i0;
+        sel1[g] = i1;
+        meta |= nib << (4 * g);
+        const uint32_t a = i0 == 0 ? w[4 * g] : (i0 == 1 ? w[4 * g + 1] : w[4 * g + 2]);
+        const uint32_t b = i1 == 3 ? w[4 * g + 3] : (i1 == 2 ? w[4 * g + 2] : w[4 * g + 1]);
+        comp[4 * g + 0] = lo16<BF16>(a);
+        comp[4 * g + 1] = hi16<BF16>(a);
+        comp[4 * g + 2] = lo16<BF16>(b);
+        comp[4 * g + 3] = hi16<BF16>(b);
+      }
+      // ---- backbone: one block of the 16 kept values
+      uint32_t bcodes[2];
+      float deq[16];
+      bsf = quant_block<FMT, 16, RESIDUAL>(comp, tc, bcodes, deq);
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.bq) + size_t(row) * (K / 4) + k0 / 4) =
+          make_uint2(bcodes[0], bcodes[1]);
+      if (RESIDUAL) {
+        // ---- residual against the quantised backbone: r = x - deq on kept pairs and
+        // x - 0 == x (exactly, -0 included) elsewhere; quantised per residual block
+#pragma unroll
+        for (int hb = 0; hb < 32 / RB; ++hb) {
+          constexpr int G = RB / 8;  // groups per residual block
+          float rv[RB];
+#pragma unroll
+          for (int gg = 0; gg < G; ++gg) {
+            const int g = hb * G + gg;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t wj = w[4 * g + j];
+              const bool f0 = sel0[g] == j, f1 = sel1[g] == j;
+              const float2 d = make_float2(f0 ? deq[4 * g] : (f1 ? deq[4 * g + 2] : 0.f),
+                                           f0 ? deq[4 * g + 1] : (f1 ? deq[4 * g + 3] : 0.f));
+              const float2 r = sub2_rn(make_float2(lo16<BF16>(wj), hi16<BF16>(wj)), d);
+              rv[8 * gg + 2 * j] = r.x;
+              rv[8 * gg + 2 * j + 1] = r.y;
+            }
+          }
+          uint32_t rcodes[RB / 8];
+          const uint32_t sfr = quant_block<FMT, RB, false>(rv, tc, rcodes, nullptr);
+          if (hb == 0) rsf0 = sfr; else rsf1 = sfr;
+          uint8_t* dst =
+              static_cast<uint8_t*>(p.rq) + size_t(row) * (K / 2) + k0 / 2 + hb * (RB / 2);
+          if constexpr (RB == 16)
+            *reinterpret_cast<uint2*>(dst) = make_uint2(rcodes[0], rcodes[1]);
+          else
+            *reinterpret_cast<uint4*>(dst) = make_uint4(rcodes[0], rcodes[1], rcodes[2], rcodes[3]);
+        }
+      }
+    }
+
+    // ---- scales and metadata: gather neighbouring lanes' bytes into 32-bit stores
+    const size_t rq32 = size_t(row & 31) * 16 + size_t((row >> 5) & 3) * 4;
+    {
+      // backbone scale column q*8+u: lanes u..u+3 form one 4-byte word
+      uint32_t word = bsf;
+      word |= __shfl_down_sync(0xFFFFFFFFu, bsf, 1) << 8;
+      word |= __shfl_down_sync(0xFFFFFFFFu, bsf, 2) << 16;
+      word |= __shfl_down_sync(0xFFFFFFFFu, bsf, 3) << 24;
+      if ((u & 3) == 0) {
+        const size_t chunk = size_t(row >> 7) * scols_b + size_t(q) * 2 + size_t(u >> 2);
+        *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.bs) + chunk * 512 + rq32) = word;
+      }
+    }
+    if (RESIDUAL) {
+      if constexpr (RB == 16) {
+        // residual scale columns q*16+2u, +1: lanes u, u+1 form one 4-byte word
+        const uint32_t two = rsf0 | (rsf1 << 8);
+        const uint32_t word = two | (__shfl_down_sync(0xFFFFFFFFu, two, 1) << 16);
+        if ((u & 1) == 0) {
+          const size_t chunk = size_t(row >> 7) * scols_r + size_t(q) * 4 + size_t(u >> 1);
+          *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.rs) + chunk * 512 + rq32) = word;
+        }
+      } else {
+        uint32_t word = rsf0;
+        word |= __shfl_down_sync(0xFFFFFFFFu, rsf0, 1) << 8;
+        word |= __shfl_down_sync(0xFFFFFFFFu, rsf0, 2) << 16;
+        word |= __shfl_down_sync(0xFFFFFFFFu, rsf0, 3) << 24;
+        if ((u & 3) == 0) {
+          const size_t chunk = size_t(row >> 7) * scols_r + size_t(q) * 2 + size_t(u >> 2);
+          *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.rs) + chunk * 512 + rq32) = word;
+        }
+      }
+    }
+    {
+      // metadata: 4 nibbles per lane, row's 16 bytes at slice q; lanes u, u+1 -> one word
+      const uint32_t m16 = meta & 0xFFFFu;
+      const uint32_t word = m16 | (__shfl_down_sync(0xFFFFFFFFu, m16, 1) << 16);
+      if ((u & 1) == 0)
+        *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.bm) + size_t(q) * Mp * 16 +
+                                     size_t(row) * 16 + u * 2) = word;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+  }
+}
+
+// ------------------------------------------------------------------------------ element 2:4
+
+// Element-wise 2:4 mask (every 4 consecutive K keep the 2 largest |x|, ties to the lower
+// index); the backbone is stored zero-filled for the dense MMA.
+
+template <bool BF16, int FMT, bool RESIDUAL>
+__global__ void __launch_bounds__(256) prep_elem_kernel(PrepParams p) {
+  constexpr int MASK = SHARQ_MASK_ELEM_2_4;
   constexpr int RB = FMT == SHARQ_NVFP4 ? 16 : 32;                  // residual block
   constexpr int BB = MASK == SHARQ_MASK_PAIR_4_8 ? 32 : RB;         // backbone block (logical)
   constexpr int CB = 256 / BB;                                       // backbone scale cols / CTA
@@ -70,10 +288,10 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
   const int k0 = q * 256 + u * 32;    // first logical K of the unit
   const int K = p.K;
 
-  float s_g = 1.f;
+  TensorConsts tc{1.f, 1.f};
   if (FMT == SHARQ_NVFP4) {
-    s_g = __fdiv_rn(__uint_as_float(*reinterpret_cast<const unsigned int*>(p.amax)), 2688.0f);
-    if (q == 0 && rb == 0 && threadIdx.x == 0) *p.tensor_scale = s_g;
+    tc = tensor_consts(__uint_as_float(*reinterpret_cast<const unsigned int*>(p.amax)));
+    if (q == 0 && rb == 0 && threadIdx.x == 0) *p.tensor_scale = tc.s_g;
   } else if (q == 0 && rb == 0 && threadIdx.x == 0) {
     *p.tensor_scale = 1.0f;
   }
@@ -111,63 +329,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     float r_val[32];  // residual before quantisation
     uint32_t meta = 0;
 
-    if (PAIR) {
-      // ---- pair-wise 4:8 mask: per group of 8, keep the 2 of 4 adjacent pairs with the
-      // largest (max |x|, min |x|), ties to the lower pair. Magnitudes compare as the
-      // 15-bit patterns of the 16-bit inputs; the pair index breaks ties.
-      float comp[16];
-      int sel0[4], sel1[4];
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t key[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t word = w[4 * g + j];
-          const uint32_t a = word & 0x7FFFu, b = (word >> 16) & 0x7FFFu;
-          key[j] = (max(a, b) << 17) | (min(a, b) << 2) | uint32_t(3 - j);
-        }
-        const int c01 = key[0] > key[1], c02 = key[0] > key[2], c03 = key[0] > key[3];
-        const int c12 = key[1] > key[2], c13 = key[1] > key[3], c23 = key[2] > key[3];
-        const bool k0p = (3 - c01 - c02 - c03) < 2;
-        const bool k1p = (c01 + 2 - c12 - c13) < 2;
-        const bool k2p = (c02 + c12 + 1 - c23) < 2;
-        const int i0 = k0p ? 0 : (k1p ? 1 : 2);
-        const int i1 = (c03 + c13 + c23) < 2 ? 3 : (k2p ? 2 : 1);
-        (void)k2p;
-        sel0[g] = i0;
-        sel1[g] = i1;
-        meta |= uint32_t(i0 | (i1 << 2)) << (4 * g);
-        const float* xg = x + 8 * g;
-        comp[4 * g + 0] = i0 == 0 ? xg[0] : (i0 == 1 ? xg[2] : xg[4]);
-        comp[4 * g + 1] = i0 == 0 ? xg[1] : (i0 == 1 ? xg[3] : xg[5]);
-        comp[4 * g + 2] = i1 == 3 ? xg[6] : (i1 == 2 ? xg[4] : xg[2]);
-        comp[4 * g + 3] = i1 == 3 ? xg[7] : (i1 == 2 ? xg[5] : xg[3]);
-      }
-      // ---- backbone: one block of the 16 kept values
-      uint32_t bcodes[2];
-      float deq[16];
-      const uint32_t bsf = quant_block<FMT, 16, RESIDUAL>(comp, s_g, bcodes, deq);
-      s_bs[tile_off(rl, u)] = uint8_t(bsf);
-      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.bq) + size_t(r) * (K / 4) + k0 / 4) =
-          make_uint2(bcodes[0], bcodes[1]);
-      *reinterpret_cast<uint16_t*>(s_bm + rl * 16 + u * 2) = uint16_t(meta);
-      if (RESIDUAL) {
-        // ---- residual against the quantised backbone
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float xv = x[8 * g + 2 * j + e];
-              const float d0 = deq[4 * g + e], d1 = deq[4 * g + 2 + e];
-              r_val[8 * g + 2 * j + e] =
-                  sel0[g] == j ? __fsub_rn(xv, d0) : (sel1[g] == j ? __fsub_rn(xv, d1) : xv);
-            }
-          }
-        }
-      }
-    } else {
+    {
       // ---- element 2:4 mask: per group of 4 keep the 2 largest |x|, ties to the lower index
       float b[32];
       uint32_t kept = 0;  // bit i: element i of the unit is on the backbone
@@ -195,12 +357,12 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
       uint32_t bcodes[4];
       float deq[32];
       if (BB == 16) {
-        const uint32_t s0 = quant_block<FMT, 16, RESIDUAL>(b, s_g, bcodes, deq);
-        const uint32_t s1 = quant_block<FMT, 16, RESIDUAL>(b + 16, s_g, bcodes + 2, deq + 16);
+        const uint32_t s0 = quant_block<FMT, 16, RESIDUAL>(b, tc, bcodes, deq);
+        const uint32_t s1 = quant_block<FMT, 16, RESIDUAL>(b + 16, tc, bcodes + 2, deq + 16);
         s_bs[tile_off(rl, 2 * u)] = uint8_t(s0);
         s_bs[tile_off(rl, 2 * u + 1)] = uint8_t(s1);
       } else {
-        const uint32_t s0 = quant_block<FMT, 32, RESIDUAL>(b, s_g, bcodes, deq);
+        const uint32_t s0 = quant_block<FMT, 32, RESIDUAL>(b, tc, bcodes, deq);
         s_bs[tile_off(rl, u)] = uint8_t(s0);
       }
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.bq) + size_t(r) * (K / 2) + k0 / 2) =
@@ -216,12 +378,12 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
     if (RESIDUAL) {
       uint32_t rcodes[4];
       if (RB == 16) {
-        const uint32_t s0 = quant_block<FMT, 16, false>(r_val, s_g, rcodes, nullptr);
-        const uint32_t s1 = quant_block<FMT, 16, false>(r_val + 16, s_g, rcodes + 2, nullptr);
+        const uint32_t s0 = quant_block<FMT, 16, false>(r_val, tc, rcodes, nullptr);
+        const uint32_t s1 = quant_block<FMT, 16, false>(r_val + 16, tc, rcodes + 2, nullptr);
         s_rs[tile_off(rl, 2 * u)] = uint8_t(s0);
         s_rs[tile_off(rl, 2 * u + 1)] = uint8_t(s1);
       } else {
-        const uint32_t s0 = quant_block<FMT, 32, false>(r_val, s_g, rcodes, nullptr);
+        const uint32_t s0 = quant_block<FMT, 32, false>(r_val, tc, rcodes, nullptr);
         s_rs[tile_off(rl, u)] = uint8_t(s0);
       }
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.rq) + size_t(r) * (K / 2) + k0 / 2) =
@@ -253,30 +415,36 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepParams p) {
 
 // ------------------------------------------------------------------------------ launch
 
-template <bool BF16, int FMT, int MASK, bool RES>
-static cudaError_t launch_prep_t(const PrepParams& p, cudaStream_t st) {
-  dim3 grid(p.K / 256, (p.M + 127) / 128);
-  prep_kernel<BF16, FMT, MASK, RES><<<grid, 256, 0, st>>>(p);
+template <bool BF16, int FMT, bool RES>
+static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
+  if (mask == SHARQ_MASK_PAIR_4_8) {
+    auto kern = prep_pair_kernel<BF16, FMT, RES>;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+    if (e != cudaSuccess) return e;
+    const long items = long(p.Mp / 4) * (p.K / 256);
+    long blocks = (items + 7) / 8;
+    const long cap = long(num_sms) * (per_sm > 0 ? per_sm : 1);
+    if (blocks > cap) blocks = cap;
+    kern<<<unsigned(blocks), 256, 0, st>>>(p);
+  } else {
+    dim3 grid(p.K / 256, (p.M + 127) / 128);
+    prep_elem_kernel<BF16, FMT, RES><<<grid, 256, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
-template <bool BF16, int FMT, int MASK>
-static cudaError_t launch_prep_r(const PrepParams& p, bool res, cudaStream_t st) {
-  return res ? launch_prep_t<BF16, FMT, MASK, true>(p, st)
-             : launch_prep_t<BF16, FMT, MASK, false>(p, st);
-}
-
 template <bool BF16, int FMT>
-static cudaError_t launch_prep_m(const PrepParams& p, int mask, bool res, cudaStream_t st) {
-  return mask == SHARQ_MASK_PAIR_4_8 ? launch_prep_r<BF16, FMT, SHARQ_MASK_PAIR_4_8>(p, res, st)
-                                     : launch_prep_r<BF16, FMT, SHARQ_MASK_ELEM_2_4>(p, res, st);
+static cudaError_t launch_prep_r(const PrepParams& p, int mask, bool res, int n, cudaStream_t st) {
+  return res ? launch_prep_t<BF16, FMT, true>(p, mask, n, st)
+             : launch_prep_t<BF16, FMT, false>(p, mask, n, st);
 }
 
 template <bool BF16>
-static cudaError_t launch_prep_f(const PrepParams& p, int fmt, int mask, bool res,
+static cudaError_t launch_prep_f(const PrepParams& p, int fmt, int mask, bool res, int n,
                                  cudaStream_t st) {
-  return fmt == SHARQ_NVFP4 ? launch_prep_m<BF16, SHARQ_NVFP4>(p, mask, res, st)
-                            : launch_prep_m<BF16, SHARQ_MXFP4>(p, mask, res, st);
+  return fmt == SHARQ_NVFP4 ? launch_prep_r<BF16, SHARQ_NVFP4>(p, mask, res, n, st)
+                            : launch_prep_r<BF16, SHARQ_MXFP4>(p, mask, res, n, st);
 }
 
 cudaError_t launch_amax(const void* X, bool bf16, size_t n_elems, unsigned int* amax_bits,
@@ -294,9 +462,9 @@ cudaError_t launch_amax(const void* X, bool bf16, size_t n_elems, unsigned int* 
 }
 
 cudaError_t launch_prep(const PrepParams& p, bool bf16, int fmt, int mask, bool residual,
-                        cudaStream_t st) {
-  return bf16 ? launch_prep_f<true>(p, fmt, mask, residual, st)
-              : launch_prep_f<false>(p, fmt, mask, residual, st);
+                        int num_sms, cudaStream_t st) {
+  return bf16 ? launch_prep_f<true>(p, fmt, mask, residual, num_sms, st)
+              : launch_prep_f<false>(p, fmt, mask, residual, num_sms, st);
 }
 
 }  // namespace sharq

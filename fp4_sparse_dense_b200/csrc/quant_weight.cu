@@ -48,10 +48,10 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(WeightQuantParams p) 
       }
     }
   }
-  float s_g = 1.f;
+  TensorConsts tc{1.f, 1.f};
   if (FMT == SHARQ_NVFP4) {
-    s_g = __fdiv_rn(p.tensor_scale[1], 2688.0f);
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) p.tensor_scale[0] = s_g;
+    tc = tensor_consts(p.tensor_scale[1]);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) p.tensor_scale[0] = tc.s_g;
   } else if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     p.tensor_scale[0] = 1.0f;
   }
@@ -66,10 +66,10 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(WeightQuantParams p) 
   uint32_t codes[4];
   uint32_t sc[2];
   if (BW == 16) {
-    sc[0] = quant_block<FMT, 16, false>(v, s_g, codes, nullptr);
-    sc[1] = quant_block<FMT, 16, false>(v + 16, s_g, codes + 2, nullptr);
+    sc[0] = quant_block<FMT, 16, false>(v, tc, codes, nullptr);
+    sc[1] = quant_block<FMT, 16, false>(v + 16, tc, codes + 2, nullptr);
   } else {
-    sc[0] = sc[1] = quant_block<FMT, 32, false>(v, s_g, codes, nullptr);
+    sc[0] = sc[1] = quant_block<FMT, 32, false>(v, tc, codes, nullptr);
   }
   *reinterpret_cast<uint4*>(p.codes + size_t(n) * (K / 2) + k0 / 2) =
       make_uint4(codes[0], codes[1], codes[2], codes[3]);

@@ -263,7 +263,7 @@ sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* a,
   p.M = a->M;
   p.K = a->K;
   p.Mp = int(round_up(size_t(a->M), 128));
-  return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, st));
+  return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
 }
 
 sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sharq_dtype y_dtype,
@@ -289,6 +289,59 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   DeviceInfo d;
   if ((s = device_info(&d)) != SHARQ_OK) return s;
   const int M = a->M, K = a->K, N = w->N;
+  GemmParams p;
+  p.bs = static_cast<const uint8_t*>(a->bs);
+  p.bm = static_cast<const uint8_t*>(a->bm);
+  p.rs = static_cast<const uint8_t*>(a->rs);
+  p.wsd = static_cast<const uint8_t*>(w->scales_dense);
+  p.wss = static_cast<const uint8_t*>(w->scales_sparse);
+  p.act_ts = a->tensor_scale;
+  p.w_ts = w->tensor_scale;
+  p.Y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.Mp = int(round_up(size_t(M), 128));
+  p.status = d.status;
+  p.timeout_ns = kWaitLimitNs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  if (M >= 256 && N % 256 == 0) {
+    // CTA-pair kernel: 256 x 256 tiles, half of the weight tile per CTA
+    const bool nv = a->cfg.fmt == SHARQ_NVFP4;
+    const uint32_t dch_rows = uint32_t(256 / (nv ? 16 : 32) / 4) * 2;  // 256-byte rows per K step
+    GemmPairMaps pm;
+    std::memset(&pm, 0, sizeof(pm));
+    if ((s = make_map(&pm.w, w->codes, uint64_t(K) / 2, uint64_t(N), 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != SHARQ_OK)
+      return s;
+    if (pair)
+      s = make_map(&pm.b, a->bq, uint64_t(K) / 4, uint64_t(M), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+    else
+      s = make_map(&pm.b, a->bq, uint64_t(K) / 2, uint64_t(M), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != SHARQ_OK) return s;
+    if (res && (s = make_map(&pm.r, a->rq, uint64_t(K) / 2, uint64_t(M), 128, 128,
+                             CU_TENSOR_MAP_SWIZZLE_128B)) != SHARQ_OK)
+      return s;
+    if (!res) pm.r = pm.b;
+    auto view = [&](CUtensorMap* mp, const void* ptr, size_t bytes, uint32_t rows) {
+      return make_map(mp, ptr, 256, uint64_t(bytes / 256), 256, rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+    };
+    if (res && (s = view(&pm.rs, a->rs, asz.rs, dch_rows)) != SHARQ_OK) return s;
+    if ((s = view(&pm.bs, a->bs, asz.bs, pair ? 4 : dch_rows)) != SHARQ_OK) return s;
+    if (pair && (s = view(&pm.bm, a->bm, asz.bm, 8)) != SHARQ_OK) return s;
+    if ((res || !pair) && (s = view(&pm.wsd, w->scales_dense, wsz.scales_dense, dch_rows)) != SHARQ_OK)
+      return s;
+    if (pair && (s = view(&pm.wss, w->scales_sparse, wsz.scales_sparse, 4)) != SHARQ_OK) return s;
+    if (!res) pm.rs = pm.bs;
+    if (!pair) pm.bm = pm.bs, pm.wss = pm.wsd;
+    if (pair && !res) pm.wsd = pm.wss;
+    p.tiles_m = (M + 127) / 128;
+    p.tiles_n = N / 256;
+    return from_cuda(launch_gemm_pair(pm, p, a->cfg.fmt, a->cfg.mask, res, y_dtype == SHARQ_F32,
+                                      d.num_sms, st));
+  }
+
   const int BN = (N % 256 == 0) ? 256 : 128;
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
@@ -304,25 +357,10 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
                            CU_TENSOR_MAP_SWIZZLE_128B)) != SHARQ_OK)
     return s;
   if (!res) maps.r = maps.b;
-  GemmParams p;
-  p.bs = static_cast<const uint8_t*>(a->bs);
-  p.bm = static_cast<const uint8_t*>(a->bm);
-  p.rs = static_cast<const uint8_t*>(a->rs);
-  p.wsd = static_cast<const uint8_t*>(w->scales_dense);
-  p.wss = static_cast<const uint8_t*>(w->scales_sparse);
-  p.act_ts = a->tensor_scale;
-  p.w_ts = w->tensor_scale;
-  p.Y = Y;
-  p.M = M;
-  p.N = N;
-  p.K = K;
-  p.Mp = int(round_up(size_t(M), 128));
   p.tiles_m = (M + 127) / 128;
   p.tiles_n = N / BN;
-  p.status = d.status;
-  p.timeout_ns = kWaitLimitNs;
   return from_cuda(launch_gemm(maps, p, a->cfg.fmt, a->cfg.mask, res, y_dtype == SHARQ_F32,
-                               d.num_sms, static_cast<cudaStream_t>(stream)));
+                               d.num_sms, st));
 }
 
 sharq_status sharq_device_status(void) {

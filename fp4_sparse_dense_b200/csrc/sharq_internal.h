@@ -5,7 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/sharq.h"
+#include "sharq.h"
 
 namespace sharq {
 
@@ -48,7 +48,7 @@ struct GemmParams {
 cudaError_t launch_amax(const void* X, bool bf16, size_t n_elems, unsigned int* amax_bits,
                         int num_sms, cudaStream_t st);
 cudaError_t launch_prep(const PrepParams& p, bool bf16, int fmt, int mask, bool residual,
-                        cudaStream_t st);
+                        int num_sms, cudaStream_t st);
 cudaError_t launch_weight_quant(const WeightQuantParams& p, bool bf16, int fmt, int mask,
                                 cudaStream_t st);
 
@@ -58,6 +58,15 @@ struct GemmMaps {
 };
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int mask,
                         bool residual, bool out_f32, int num_sms, cudaStream_t st);
+
+// maps of the CTA-pair kernel: the three FP4 operands plus byte views [bytes/256][256] of
+// the scale and metadata buffers (loaded by tensor copies so that both CTAs can count them
+// on the pair leader's barrier)
+struct GemmPairMaps {
+  CUtensorMap w, b, r, rs, bs, bm, wsd, wss;
+};
+cudaError_t launch_gemm_pair(const GemmPairMaps& maps, const GemmParams& p, int fmt, int mask,
+                             bool residual, bool out_f32, int num_sms, cudaStream_t st);
 
 // block sizes along K
 inline int residual_block(int fmt) { return fmt == SHARQ_NVFP4 ? 16 : 32; }

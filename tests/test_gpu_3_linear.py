@@ -51,6 +51,15 @@ GEMM_CASES = [
     ("nvfp4", "elem24", True, 130, 512, 256),
     ("nvfp4", "elem24", False, 64, 256, 128),
 ]
+PAIR_CASES = [  # M >= 256 and N % 256 == 0: the CTA-pair kernel (odd 128-row counts included)
+    ("nvfp4", "pair48", True, 256, 512, 256),
+    ("nvfp4", "pair48", True, 300, 1024, 512),
+    ("nvfp4", "pair48", True, 640, 768, 768),
+    ("nvfp4", "pair48", False, 512, 256, 256),
+    ("nvfp4", "elem24", True, 384, 512, 256),
+    ("mxfp4", "pair48", True, 513, 512, 256),
+    ("mxfp4", "elem24", True, 256, 256, 512),
+]
 MX_CASES = [
     ("mxfp4", "pair48", True, 128, 512, 256),
     ("mxfp4", "pair48", True, 77, 1024, 128),
@@ -59,7 +68,7 @@ MX_CASES = [
 ]
 
 
-@pytest.mark.parametrize("fmt,mask,residual,M,K,N", GEMM_CASES + MX_CASES)
+@pytest.mark.parametrize("fmt,mask,residual,M,K,N", GEMM_CASES + MX_CASES + PAIR_CASES)
 @pytest.mark.parametrize("out_f32", [True, False])
 def test_gemm_on_oracle_operands(fmt, mask, residual, M, K, N, out_f32):
     """The GEMM alone: operands are the oracle's bytes uploaded to the GPU."""
@@ -74,7 +83,7 @@ def test_gemm_on_oracle_operands(fmt, mask, residual, M, K, N, out_f32):
     check_y(gpu_linear(act, wt, out_f32), S.linear(p, qw), not out_f32)
 
 
-@pytest.mark.parametrize("fmt,mask,residual,M,K,N", GEMM_CASES + MX_CASES)
+@pytest.mark.parametrize("fmt,mask,residual,M,K,N", GEMM_CASES + MX_CASES + PAIR_CASES)
 def test_end_to_end(fmt, mask, residual, M, K, N):
     """prepare + quantize_weight + linear on the GPU vs the oracle chain."""
     import fp4_sparse_dense_b200 as sq
