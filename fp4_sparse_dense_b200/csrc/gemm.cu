@@ -26,6 +26,7 @@
 #include <cuda_runtime.h>
 
 #include "sharq_internal.h"
+#include "epilogue.cuh"
 #include "sm100_ptx.cuh"
 
 namespace sharq {
@@ -60,9 +61,11 @@ struct GemmCfg {
   static constexpr int STAGE_RAW = OFF_E + E_BYTES;
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int TX = STAGE_RAW;  // every byte of the stage arrives by copy
-  static constexpr int STAGES_FIT = (kMaxSmem - 2048) / STAGE;
+  static constexpr int EPI_BYTES = 8 * 2048;  // one 32 x 32 bf16 staging box per epilogue warp
+  static constexpr int STAGES_FIT = (kMaxSmem - 2048 - EPI_BYTES) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static constexpr int SMEM = STAGES * STAGE + 2048;  // + alignment slack and barriers
+  // stages, 1 KB of barriers, the epilogue staging, 1 KB alignment slack
+  static constexpr int SMEM = STAGES * STAGE + 1024 + EPI_BYTES + 1024;
   // tensor-memory columns
   static constexpr int COL_SFR = 256;
   static constexpr int COL_SFB = COL_SFR + (RES ? DCH * 4 : 0);
@@ -84,7 +87,8 @@ template <int FMT, bool PAIR, bool RES, int BN, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
     sharq_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_b,
-                      const __grid_constant__ CUtensorMap tm_r, const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tm_r,
+                      const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   using C = GemmCfg<FMT, PAIR, RES, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -297,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const float alpha = __fmul_rn(p.act_ts[0], p.w_ts[0]);
+    const uint32_t epi_stage = ptx::smem_u32(ctrl + 1024 + (warp - 2) * 2048);
     int tcount = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
@@ -314,33 +319,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tmem_ld_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_u32(tempty_bar));
-      if (row < p.M) {
-        const size_t off = size_t(row) * p.N + size_t(nb) * BN + size_t(half) * HALF;
-        if (OUT_F32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + off);
-#pragma unroll
-          for (int i = 0; i < HALF / 4; ++i)
-            dst[i] = make_float4(__fmul_rn(__uint_as_float(v[4 * i]), alpha),
-                                 __fmul_rn(__uint_as_float(v[4 * i + 1]), alpha),
-                                 __fmul_rn(__uint_as_float(v[4 * i + 2]), alpha),
-                                 __fmul_rn(__uint_as_float(v[4 * i + 3]), alpha));
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + off);
-#pragma unroll
-          for (int i = 0; i < HALF / 8; ++i) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const __nv_bfloat162 b2 =
-                  __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[8 * i + 2 * h]), alpha),
-                                        __fmul_rn(__uint_as_float(v[8 * i + 2 * h + 1]), alpha));
-              w4[h] = *reinterpret_cast<const uint32_t*>(&b2);
-            }
-            dst[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-        }
-      }
+      if (OUT_F32)
+        store_rows_f32<HALF>(static_cast<float*>(p.Y), p.M, p.N, v, alpha, row, nb * BN + half * HALF);
+      else
+        store_rows_bf16<HALF>(&tm_y, epi_stage, v, alpha, mb * 128 + quarter * 32, nb * BN + half * HALF, lane);
     }
+    if (!OUT_F32 && lane == 0) ptx::bulk_wait_all();  // stores complete before exit
     if (!ok && lane == 0) atomicExch(p.status, unsigned(SHARQ_ERR_TIMEOUT));
   }
 
@@ -360,7 +344,7 @@ static cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, int num_sms,
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  kern<<<grid, kThreads, C::SMEM, st>>>(m.w, m.b, m.r, p);
+  kern<<<grid, kThreads, C::SMEM, st>>>(m.w, m.b, m.r, m.y, p);
   return cudaGetLastError();
 }
 

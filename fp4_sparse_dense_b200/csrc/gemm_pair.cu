@@ -9,7 +9,7 @@
 // is bound by L2 -> SM traffic at prefill sizes).
 //
 // Protocol (leader = cluster rank 0):
-//   * every load of both CTAs (FP4 tiles, scales, metadata; all 2-D tensor maps) counts
+//   * every load of both CTAs (FP4 tiles, scales, metadata; all tensor maps) counts
 //     its bytes on the leader's `full` barrier of the stage; the leader arms it for the
 //     bytes of both CTAs;
 //   * the leader's single MMA thread copies scales / metadata into both CTAs' tensor
@@ -24,6 +24,7 @@
 #include <cuda_runtime.h>
 
 #include "sharq_internal.h"
+#include "epilogue.cuh"
 #include "sm100_ptx.cuh"
 
 namespace sharq {
@@ -61,9 +62,11 @@ struct PairCfg {
   static constexpr int STAGE_RAW = OFF_E + E_BYTES;
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int TX_PAIR = 2 * STAGE_RAW;  // bytes of both CTAs, counted by the leader
-  static constexpr int STAGES_FIT = (kPairMaxSmem - 2048) / STAGE;
+  static constexpr int EPI_BYTES = kPairEpiWarps * 2048;  // 32 x 32 bf16 box per warp
+  static constexpr int STAGES_FIT = (kPairMaxSmem - 2048 - EPI_BYTES) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int SMEM = STAGES * STAGE + 2048;
+  // stages, 1 KB of barriers, the epilogue staging, 1 KB alignment slack
+  static constexpr int SMEM = STAGES * STAGE + 1024 + EPI_BYTES + 1024;
   // tensor-memory columns (same in both CTAs)
   static constexpr int COL_SFR = 256;
   static constexpr int COL_SFB = COL_SFR + (RES ? DCH * 4 : 0);
@@ -166,17 +169,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             ptx::tma_load_2d_pair(st + C::OFF_SFB, &m.bs, 0, (rb_sf * (p.K / 128) + kt * 2) * 2, fb);
             ptx::tma_load_2d_pair(st + C::OFF_E, &m.bm, 0,
                                   (kt * p.Mp * 16 + rb_sf * 2048) / 256, fb);
-            for (int h = 0; h < 2; ++h)
-              ptx::tma_load_2d_pair(st + C::OFF_SWS + h * 1024, &m.wss, 0,
-                                    ((nb * 2 + h) * (p.K / 128) + kt * 2) * 2, fb);
+            // both 128-row halves of the weight tile's sparse-view scales in one box
+            ptx::tma_load_4d_pair(st + C::OFF_SWS, &m.wss, 0, 0, kt, nb * 2, fb);
           } else {
             ptx::tma_load_2d_pair(st + C::OFF_SFB, &m.bs, 0,
                                   (rb_sf * (p.K / C::GD / 4) + kt * C::DCH) * 2, fb);
           }
-          if (C::DENSE_W)
-            for (int h = 0; h < 2; ++h)
-              ptx::tma_load_2d_pair(st + C::OFF_SWD + h * C::DCH * 512, &m.wsd, 0,
-                                    ((nb * 2 + h) * (p.K / C::GD / 4) + kt * C::DCH) * 2, fb);
+          if (C::DENSE_W)  // both halves of the dense-view weight scales in one box
+            ptx::tma_load_4d_pair(st + C::OFF_SWD, &m.wsd, 0, 0, kt, nb * 2, fb);
           if (++s == C::STAGES) { s = 0; ph ^= 1u; }
         }
       }
@@ -294,6 +294,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const float alpha = __fmul_rn(p.act_ts[0], p.w_ts[0]);
+    const uint32_t epi_stage = ptx::smem_u32(ctrl + 1024 + (warp - 2) * 2048);
     int tcount = 0;
     bool ok = true;
     for (int t = cluster; t < pair_tiles; t += n_clusters, ++tcount) {
@@ -312,33 +313,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(lead_tempty);
-      if (row < p.M) {
-        const size_t off = size_t(row) * p.N + size_t(nb) * C::BN + size_t(half) * HALF;
-        if (OUT_F32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + off);
-#pragma unroll
-          for (int i = 0; i < HALF / 4; ++i)
-            dst[i] = make_float4(__fmul_rn(__uint_as_float(v[4 * i]), alpha),
-                                 __fmul_rn(__uint_as_float(v[4 * i + 1]), alpha),
-                                 __fmul_rn(__uint_as_float(v[4 * i + 2]), alpha),
-                                 __fmul_rn(__uint_as_float(v[4 * i + 3]), alpha));
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + off);
-#pragma unroll
-          for (int i = 0; i < HALF / 8; ++i) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const __nv_bfloat162 b2 =
-                  __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[8 * i + 2 * h]), alpha),
-                                        __fmul_rn(__uint_as_float(v[8 * i + 2 * h + 1]), alpha));
-              w4[h] = *reinterpret_cast<const uint32_t*>(&b2);
-            }
-            dst[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-        }
-      }
+      if (OUT_F32)
+        store_rows_f32<HALF>(static_cast<float*>(p.Y), p.M, p.N, v, alpha, row, nb * C::BN + half * HALF);
+      else
+        store_rows_bf16<HALF>(&m.y, epi_stage, v, alpha, (mb2 * 2 + int(rank)) * 128 + quarter * 32, nb * C::BN + half * HALF, lane);
     }
+    if (!OUT_F32 && lane == 0) ptx::bulk_wait_all();  // stores complete before exit
     if (!ok && lane == 0) atomicExch(p.status, unsigned(SHARQ_ERR_TIMEOUT));
   }
 

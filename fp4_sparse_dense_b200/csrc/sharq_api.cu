@@ -93,29 +93,46 @@ EncodeTiledFn encode_fn() {
 
 struct MapKey {
   const void* ptr;
-  uint64_t inner, rows;
-  uint32_t box_inner, box_rows, swz;
+  int rank, dtype, swz;
+  uint64_t dims[4], strides[3];
+  uint32_t box[4];
   bool operator==(const MapKey& o) const {
-    return ptr == o.ptr && inner == o.inner && rows == o.rows && box_inner == o.box_inner &&
-           box_rows == o.box_rows && swz == o.swz;
+    if (ptr != o.ptr || rank != o.rank || dtype != o.dtype || swz != o.swz) return false;
+    for (int i = 0; i < 4; ++i)
+      if (dims[i] != o.dims[i] || box[i] != o.box[i]) return false;
+    for (int i = 0; i < 3; ++i)
+      if (strides[i] != o.strides[i]) return false;
+    return true;
   }
 };
 struct MapKeyHash {
   size_t operator()(const MapKey& k) const {
-    size_t h = reinterpret_cast<size_t>(k.ptr);
-    h ^= (k.inner * 0x9E3779B97F4A7C15ull) + (h << 6) + (h >> 2);
-    h ^= (k.rows * 0xC2B2AE3D27D4EB4Full) + (h << 6) + (h >> 2);
-    h ^= (uint64_t(k.box_inner) << 32 | uint64_t(k.box_rows) << 8 | k.swz) + (h << 6) + (h >> 2);
-    return h;
+    uint64_t h = reinterpret_cast<uint64_t>(k.ptr) * 0x9E3779B97F4A7C15ull;
+    auto mix = [&](uint64_t v) { h ^= v + 0x9E3779B97F4A7C15ull + (h << 6) + (h >> 2); };
+    mix(uint64_t(k.rank) | uint64_t(k.dtype) << 8 | uint64_t(k.swz) << 16);
+    for (int i = 0; i < 4; ++i) mix(k.dims[i] ^ (uint64_t(k.box[i]) << 40));
+    for (int i = 0; i < 3; ++i) mix(k.strides[i]);
+    return size_t(h);
   }
 };
 std::mutex g_map_mu;
 std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
 
-// 2-D byte matrix [rows][inner] (row pitch = inner), box [box_rows][box_inner]
-sharq_status make_map(CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t rows,
-                      uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
-  MapKey key{ptr, inner, rows, box_inner, box_rows, uint32_t(swz)};
+// Tensor map of a `rank`-dimensional tensor: dims in elements (innermost first), strides
+// in bytes of dimensions 1..rank-1, box in elements. Cached by (pointer, shape).
+sharq_status make_map_nd(CUtensorMap* out, const void* ptr, CUtensorMapDataType dtype, int rank,
+                         const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                         CUtensorMapSwizzle swz) {
+  MapKey key{};
+  key.ptr = ptr;
+  key.rank = rank;
+  key.dtype = int(dtype);
+  key.swz = int(swz);
+  for (int i = 0; i < rank; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+    if (i > 0) key.strides[i - 1] = strides[i - 1];
+  }
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -126,18 +143,50 @@ sharq_status make_map(CUtensorMap* out, const void* ptr, uint64_t inner, uint64_
   }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return SHARQ_ERR_CUDA;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner};
-  cuuint32_t box[2] = {box_inner, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  cuuint64_t d[4], st[3];
+  cuuint32_t b[4], es[4] = {1, 1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    if (i > 0) st[i - 1] = strides[i - 1];
+  }
+  CUresult r = fn(out, dtype, cuuint32_t(rank), const_cast<void*>(ptr), d, st, b, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return SHARQ_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_map_mu);
   if (g_maps.size() > 4096) g_maps.clear();
   g_maps[key] = *out;
   return SHARQ_OK;
+}
+
+// 2-D byte matrix [rows][inner] (row pitch = inner), box [box_rows][box_inner]
+sharq_status make_map(CUtensorMap* out, const void* ptr, uint64_t inner, uint64_t rows,
+                      uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  const uint64_t dims[2] = {inner, rows};
+  const uint64_t strides[1] = {inner};
+  const uint32_t box[2] = {box_inner, box_rows};
+  return make_map_nd(out, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, dims, strides, box, swz);
+}
+
+// bf16 output Y[M][N]: 32 x 32 boxes with the 64-byte swizzle of the epilogue staging
+sharq_status make_y_map(CUtensorMap* out, const void* Y, int M, int N) {
+  const uint64_t dims[2] = {uint64_t(N), uint64_t(M)};
+  const uint64_t strides[1] = {uint64_t(N) * 2};
+  const uint32_t box[2] = {32, 32};
+  return make_map_nd(out, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// weight scales seen as [N/128 row blocks][K/256 steps][rows_per_step][256 bytes], so that
+// one box fetches the chunks of both 128-row halves of a 256-row tile for one K step
+sharq_status make_wscale_map(CUtensorMap* out, const void* ptr, int K, int N, uint32_t rows_per_step) {
+  const uint64_t KT = uint64_t(K) / 256;
+  const uint64_t dims[4] = {256, rows_per_step, KT, uint64_t(N) / 128};
+  const uint64_t strides[3] = {256, uint64_t(rows_per_step) * 256, KT * rows_per_step * 256};
+  const uint32_t box[4] = {256, rows_per_step, 1, 2};
+  return make_map_nd(out, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 sharq_status act_sizes(int32_t M, int32_t K, sharq_config c, sharq_act_bytes* o) {
@@ -330,9 +379,11 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
     if (res && (s = view(&pm.rs, a->rs, asz.rs, dch_rows)) != SHARQ_OK) return s;
     if ((s = view(&pm.bs, a->bs, asz.bs, pair ? 4 : dch_rows)) != SHARQ_OK) return s;
     if (pair && (s = view(&pm.bm, a->bm, asz.bm, 8)) != SHARQ_OK) return s;
-    if ((res || !pair) && (s = view(&pm.wsd, w->scales_dense, wsz.scales_dense, dch_rows)) != SHARQ_OK)
+    if ((res || !pair) &&
+        (s = make_wscale_map(&pm.wsd, w->scales_dense, K, N, dch_rows)) != SHARQ_OK)
       return s;
-    if (pair && (s = view(&pm.wss, w->scales_sparse, wsz.scales_sparse, 4)) != SHARQ_OK) return s;
+    if (pair && (s = make_wscale_map(&pm.wss, w->scales_sparse, K, N, 4)) != SHARQ_OK) return s;
+    if (y_dtype == SHARQ_BF16 && (s = make_y_map(&pm.y, Y, M, N)) != SHARQ_OK) return s;
     if (!res) pm.rs = pm.bs;
     if (!pair) pm.bm = pm.bs, pm.wss = pm.wsd;
     if (pair && !res) pm.wsd = pm.wss;
@@ -357,6 +408,7 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
                            CU_TENSOR_MAP_SWIZZLE_128B)) != SHARQ_OK)
     return s;
   if (!res) maps.r = maps.b;
+  if (y_dtype == SHARQ_BF16 && (s = make_y_map(&maps.y, Y, M, N)) != SHARQ_OK) return s;
   p.tiles_m = (M + 127) / 128;
   p.tiles_n = N / BN;
   return from_cuda(launch_gemm(maps, p, a->cfg.fmt, a->cfg.mask, res, y_dtype == SHARQ_F32,

@@ -54,7 +54,7 @@ cudaError_t launch_weight_quant(const WeightQuantParams& p, bool bf16, int fmt, 
 
 // maps for the three FP4 operands, built by the host side
 struct GemmMaps {
-  CUtensorMap w, b, r;
+  CUtensorMap w, b, r, y;  // y: bf16 output, 32 x 32 boxes (unused for float output)
 };
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int mask,
                         bool residual, bool out_f32, int num_sms, cudaStream_t st);
@@ -63,7 +63,7 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int 
 // the scale and metadata buffers (loaded by tensor copies so that both CTAs can count them
 // on the pair leader's barrier)
 struct GemmPairMaps {
-  CUtensorMap w, b, r, rs, bs, bm, wsd, wss;
+  CUtensorMap w, b, r, rs, bs, bm, wsd, wss, y;
 };
 cudaError_t launch_gemm_pair(const GemmPairMaps& maps, const GemmParams& p, int fmt, int mask,
                              bool residual, bool out_f32, int num_sms, cudaStream_t st);
