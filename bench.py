@@ -226,6 +226,7 @@ def run_gpu(args):
     QW = [sq.quantize_weight(w) for w in W]
     ACT = [sq.empty_act(M, K, cfg, dev) for _ in range(n_sets)]
     Y = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(n_sets)]
+    WS = sq.linear_workspace(M, N, K, cfg, dev)  # split-K scratch (None for prefill shapes)
     stream = torch.cuda.current_stream()
 
     def step(i):
@@ -233,7 +234,7 @@ def run_gpu(args):
         return a
 
     for i in range(args.warmup):
-        sq.linear(step(i), QW[i % 2], out=Y[i % n_sets])
+        sq.linear(step(i), QW[i % 2], out=Y[i % n_sets], workspace=WS)
     torch.cuda.synchronize()
     status = sq.sharq_device_status()
     assert status == 0, sq.sharq_status_string(status)
@@ -251,7 +252,7 @@ def run_gpu(args):
             ev[i][0].record(stream)
             a = step(i)
             ev[i][1].record(stream)
-            sq.linear(a, QW[i % 2], out=Y[i % n_sets])
+            sq.linear(a, QW[i % 2], out=Y[i % n_sets], workspace=WS)
             ev[i][2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -276,7 +277,7 @@ def run_gpu(args):
     for i in range(e2e_steps):
         X[i % n_sets].copy_(xh[i % n_sets], non_blocking=True)
         a = step(i)
-        sq.linear(a, QW[i % 2], out=Y[i % n_sets])
+        sq.linear(a, QW[i % 2], out=Y[i % n_sets], workspace=WS)
         yh.copy_(Y[i % n_sets], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()

@@ -19,13 +19,14 @@ from ._abi import (  # noqa: F401
     ELEM_2_4, F16, F32, BF16, MXFP4, NVFP4, PAIR_4_8, SharqError, lib, lib_path,
     sharq_act, sharq_act_bytes, sharq_config, sharq_weight, sharq_weight_bytes, check,
     sharq_act_sizes, sharq_weight_sizes, sharq_status_string, sharq_device_status,
-    sharq_prepare, sharq_quantize_weight, sharq_linear,
+    sharq_prepare, sharq_quantize_weight, sharq_linear, sharq_linear_workspace_size,
 )
 
 __all__ = [
     "Config", "QuantWeight", "PreparedAct", "quantize_weight", "prepare", "linear",
     "sharq_act_sizes", "sharq_weight_sizes", "sharq_prepare", "sharq_quantize_weight",
-    "sharq_linear", "sharq_device_status", "sharq_status_string", "SharqError",
+    "sharq_linear", "sharq_linear_workspace_size", "sharq_device_status",
+    "sharq_status_string", "SharqError", "linear_workspace",
     "NVFP4", "MXFP4", "PAIR_4_8", "ELEM_2_4", "F16", "BF16", "F32",
 ]
 
@@ -147,13 +148,30 @@ def prepare(X, cfg: Config = Config(), out: PreparedAct | None = None, stream=No
     return out
 
 
-def linear(act: PreparedAct, w: QuantWeight, out=None, out_dtype=None, stream=None):
-    """Y[M x N] = sparse-FP4-GEMM(backbone, W) + dense-FP4-GEMM(residual, W)."""
+def linear_workspace(M: int, N: int, K: int, cfg: Config = Config(), device="cuda"):
+    """Caller-owned split-K workspace for sharq_linear (None when the shape does not split)."""
+    nbytes = ctypes.c_size_t(0)
+    check(sharq_linear_workspace_size(M, N, K, cfg.c(), ctypes.byref(nbytes)))
+    return _u8(nbytes.value, device) if nbytes.value else None
+
+
+def linear(act: PreparedAct, w: QuantWeight, out=None, out_dtype=None, workspace="auto",
+           stream=None):
+    """Y[M x N] = sparse-FP4-GEMM(backbone, W) + dense-FP4-GEMM(residual, W).
+
+    workspace: "auto" allocates the split-K workspace this shape wants (a torch buffer the
+    caller may keep and pass again), None runs without splitting K, or a uint8 CUDA tensor.
+    """
     torch = _torch()
     out_dtype = out_dtype or torch.bfloat16
     if out is None:
         out = torch.empty(act.M, w.N, dtype=out_dtype, device=act.bq.device)
     code = {torch.bfloat16: BF16, torch.float32: F32}[out.dtype]
+    if isinstance(workspace, str):
+        workspace = linear_workspace(act.M, w.N, act.K, act.cfg, act.bq.device)
+    ws_ptr = _ptr(workspace)
+    ws_bytes = workspace.numel() if workspace is not None else 0
     ca, cw = act.c(), w.c()
-    check(sharq_linear(ctypes.byref(ca), ctypes.byref(cw), _ptr(out), code, _stream(stream)))
+    check(sharq_linear(ctypes.byref(ca), ctypes.byref(cw), _ptr(out), code, ws_ptr, ws_bytes,
+                       _stream(stream)))
     return out

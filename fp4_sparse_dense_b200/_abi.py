@@ -62,7 +62,9 @@ def _load():
         "sharq_quantize_weight": (st, [vp, ctypes.c_int, ctypes.POINTER(sharq_weight), vp]),
         "sharq_prepare": (st, [vp, ctypes.c_int, ctypes.POINTER(sharq_act), vp]),
         "sharq_linear": (st, [ctypes.POINTER(sharq_act), ctypes.POINTER(sharq_weight), vp,
-                              ctypes.c_int, vp]),
+                              ctypes.c_int, vp, ctypes.c_size_t, vp]),
+        "sharq_linear_workspace_size": (st, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                             sharq_config, ctypes.POINTER(ctypes.c_size_t)]),
         "sharq_device_status": (st, []),
         "sharq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
@@ -79,6 +81,7 @@ sharq_weight_sizes = lib.sharq_weight_sizes
 sharq_quantize_weight = lib.sharq_quantize_weight
 sharq_prepare = lib.sharq_prepare
 sharq_linear = lib.sharq_linear
+sharq_linear_workspace_size = lib.sharq_linear_workspace_size
 sharq_device_status = lib.sharq_device_status
 sharq_status_string = lib.sharq_status_string
 

@@ -105,7 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int KT = p.K / 256;
-  const int tiles = p.tiles_m * p.tiles_n;
+  const int tiles_mn = p.tiles_m * p.tiles_n;
+  const int tiles = tiles_mn * p.splits;  // split-K: `splits` K ranges per output tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -140,8 +141,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        const int mb = t % p.tiles_m, nb = t / p.tiles_m;
-        for (int kt = 0; kt < KT; ++kt) {
+        const int tmn = t % tiles_mn, ks = t / tiles_mn;
+        const int mb = tmn % p.tiles_m, nb = tmn / p.tiles_m;
+        const int kt0 = ks * KT / p.splits, kt1 = (ks + 1) * KT / p.splits;
+        for (int kt = kt0; kt < kt1; ++kt) {
           if (!ptx::mbar_wait(ptx::smem_u32(empty_bar + s), ph ^ 1u, abort_flag, limit)) {
             ok = false;
             break;
@@ -202,7 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ptx::tc_fence_after();
         }
-        for (int kt = 0; kt < KT; ++kt) {
+        const int ks = t / tiles_mn;
+        const int kt0 = ks * KT / p.splits, kt1 = (ks + 1) * KT / p.splits;
+        for (int kt = kt0; kt < kt1; ++kt) {
           if (!ptx::mbar_wait(ptx::smem_u32(full_bar + s), ph, abort_flag, limit)) {
             ok = false;
             break;
@@ -240,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::smem_desc(st + C::OFF_SWD + (rb * C::DCH + c) * 512, 16, 128, 0));
           }
           // ---- MMAs: backbone then residual, one accumulator
-          uint32_t acc = kt > 0 ? 1u : 0u;
+          uint32_t acc = kt > kt0 ? 1u : 0u;
           if (PAIR) {
             for (int j = 0; j < 2; ++j) {
               const uint64_t a = ptx::smem_desc(st + C::OFF_B + 32 * j, 16, 512, 4);
@@ -305,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tcount = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
-      const int mb = t % p.tiles_m, nb = t / p.tiles_m;
+      const int tmn = t % tiles_mn, ks = t / tiles_mn;
+      const int mb = tmn % p.tiles_m, nb = tmn / p.tiles_m;
       if (!ptx::mbar_wait(ptx::smem_u32(tfull_bar), uint32_t(tcount) & 1u, abort_flag, limit)) {
         ok = false;
         break;
@@ -319,12 +325,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tmem_ld_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_u32(tempty_bar));
-      if (OUT_F32)
+      if (p.splits > 1)  // unscaled FP32 partial of this K range, reduced by a second kernel
+        store_rows_f32<HALF>(p.ws + size_t(ks) * p.M * p.N, p.M, p.N, v, 1.0f, row,
+                             nb * BN + half * HALF);
+      else if (OUT_F32)
         store_rows_f32<HALF>(static_cast<float*>(p.Y), p.M, p.N, v, alpha, row, nb * BN + half * HALF);
       else
         store_rows_bf16<HALF>(&tm_y, epi_stage, v, alpha, mb * 128 + quarter * 32, nb * BN + half * HALF, lane);
     }
-    if (!OUT_F32 && lane == 0) ptx::bulk_wait_all();  // stores complete before exit
+    if (!OUT_F32 && p.splits == 1 && lane == 0) ptx::bulk_wait_all();  // stores done before exit
     if (!ok && lane == 0) atomicExch(p.status, unsigned(SHARQ_ERR_TIMEOUT));
   }
 
@@ -342,10 +351,55 @@ static cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, int num_sms,
   auto kern = sharq_gemm_kernel<FMT, PAIR, RES, BN, OUT_F32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  const int tiles = p.tiles_m * p.tiles_n;
+  const int tiles = p.tiles_m * p.tiles_n * p.splits;
   const int grid = tiles < num_sms ? tiles : num_sms;
   kern<<<grid, kThreads, C::SMEM, st>>>(m.w, m.b, m.r, m.y, p);
   return cudaGetLastError();
+}
+
+// Split-K reduction: Y = alpha * sum over the K ranges of the FP32 partials, in a fixed
+// order (deterministic). One thread per 8 consecutive outputs.
+template <bool OUT_F32>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ ws,
+                                                            int splits, int M, int N,
+                                                            const float* act_ts, const float* w_ts,
+                                                            void* Y) {
+  const size_t total = size_t(M) * N;
+  const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (i >= total) return;
+  const float alpha = __fmul_rn(act_ts[0], w_ts[0]);
+  float acc[8];
+  {
+    const float4 a = *reinterpret_cast<const float4*>(ws + i);
+    const float4 b = *reinterpret_cast<const float4*>(ws + i + 4);
+    acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+    acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+  }
+  for (int sidx = 1; sidx < splits; ++sidx) {
+    const float* src = ws + size_t(sidx) * total + i;
+    const float4 a = *reinterpret_cast<const float4*>(src);
+    const float4 b = *reinterpret_cast<const float4*>(src + 4);
+    acc[0] = __fadd_rn(acc[0], a.x); acc[1] = __fadd_rn(acc[1], a.y);
+    acc[2] = __fadd_rn(acc[2], a.z); acc[3] = __fadd_rn(acc[3], a.w);
+    acc[4] = __fadd_rn(acc[4], b.x); acc[5] = __fadd_rn(acc[5], b.y);
+    acc[6] = __fadd_rn(acc[6], b.z); acc[7] = __fadd_rn(acc[7], b.w);
+  }
+  if (OUT_F32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(Y) + i);
+    dst[0] = make_float4(__fmul_rn(acc[0], alpha), __fmul_rn(acc[1], alpha),
+                         __fmul_rn(acc[2], alpha), __fmul_rn(acc[3], alpha));
+    dst[1] = make_float4(__fmul_rn(acc[4], alpha), __fmul_rn(acc[5], alpha),
+                         __fmul_rn(acc[6], alpha), __fmul_rn(acc[7], alpha));
+  } else {
+    uint32_t w4[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(acc[2 * h], alpha),
+                                                      __fmul_rn(acc[2 * h + 1], alpha));
+      w4[h] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(Y) + i) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
 }
 
 template <int FMT, bool PAIR, bool RES, int BN>
@@ -376,8 +430,17 @@ static cudaError_t launch_m(const GemmMaps& m, const GemmParams& p, int mask, bo
 
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int mask,
                         bool residual, bool out_f32, int num_sms, cudaStream_t st) {
-  return fmt == SHARQ_NVFP4 ? launch_m<SHARQ_NVFP4>(maps, p, mask, residual, out_f32, num_sms, st)
-                            : launch_m<SHARQ_MXFP4>(maps, p, mask, residual, out_f32, num_sms, st);
+  cudaError_t e =
+      fmt == SHARQ_NVFP4 ? launch_m<SHARQ_NVFP4>(maps, p, mask, residual, out_f32, num_sms, st)
+                         : launch_m<SHARQ_MXFP4>(maps, p, mask, residual, out_f32, num_sms, st);
+  if (e != cudaSuccess || p.splits <= 1) return e;
+  const size_t total = size_t(p.M) * p.N;
+  const unsigned blocks = unsigned((total / 8 + 255) / 256);
+  if (out_f32)
+    splitk_reduce_kernel<true><<<blocks, 256, 0, st>>>(p.ws, p.splits, p.M, p.N, p.act_ts, p.w_ts, p.Y);
+  else
+    splitk_reduce_kernel<false><<<blocks, 256, 0, st>>>(p.ws, p.splits, p.M, p.N, p.act_ts, p.w_ts, p.Y);
+  return cudaGetLastError();
 }
 
 }  // namespace sharq

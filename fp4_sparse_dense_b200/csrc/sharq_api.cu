@@ -315,8 +315,23 @@ sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* a,
   return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
 }
 
+sharq_status sharq_linear_workspace_size(int32_t M, int32_t N, int32_t K, sharq_config cfg,
+                                         size_t* bytes) {
+  if (!bytes) return SHARQ_ERR_INVALID_ARG;
+  sharq_act_bytes asz;
+  sharq_weight_bytes wsz;
+  sharq_status s = act_sizes(M, K, cfg, &asz);
+  if (s != SHARQ_OK) return s;
+  if ((s = weight_sizes(K, N, cfg, &wsz)) != SHARQ_OK) return s;
+  DeviceInfo d;
+  if ((s = device_info(&d)) != SHARQ_OK) return s;
+  const int splits = plan_splits(M, N, K, d.num_sms);
+  *bytes = splits > 1 ? size_t(splits) * size_t(M) * size_t(N) * sizeof(float) : 0;
+  return SHARQ_OK;
+}
+
 sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sharq_dtype y_dtype,
-                          void* stream) {
+                          void* workspace, size_t workspace_bytes, void* stream) {
   if (!a || !w || !Y) return SHARQ_ERR_INVALID_ARG;
   if (y_dtype != SHARQ_BF16 && y_dtype != SHARQ_F32) return SHARQ_ERR_INVALID_ARG;
   if (std::memcmp(&a->cfg, &w->cfg, sizeof(sharq_config)) != 0 || a->K != w->K)
@@ -353,6 +368,8 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   p.Mp = int(round_up(size_t(M), 128));
   p.status = d.status;
   p.timeout_ns = kWaitLimitNs;
+  p.splits = 1;
+  p.ws = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   if (M >= 256 && N % 256 == 0) {
@@ -409,6 +426,14 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
     return s;
   if (!res) maps.r = maps.b;
   if (y_dtype == SHARQ_BF16 && (s = make_y_map(&maps.y, Y, M, N)) != SHARQ_OK) return s;
+  {
+    const int splits = plan_splits(M, N, K, d.num_sms);
+    const size_t need = size_t(splits) * size_t(M) * size_t(N) * sizeof(float);
+    if (splits > 1 && workspace && workspace_bytes >= need && aligned16(workspace)) {
+      p.splits = splits;
+      p.ws = static_cast<float*>(workspace);
+    }
+  }
   p.tiles_m = (M + 127) / 128;
   p.tiles_n = N / BN;
   return from_cuda(launch_gemm(maps, p, a->cfg.fmt, a->cfg.mask, res, y_dtype == SHARQ_F32,

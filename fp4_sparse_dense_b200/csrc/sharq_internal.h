@@ -41,6 +41,8 @@ struct GemmParams {
   void* Y;
   int M, N, K, Mp;
   int tiles_m, tiles_n;
+  int splits;  // K ranges per output tile (1: no split; >1: partials in ws, then a reduction)
+  float* ws;   // split-K partials [splits][M][N] (caller-owned workspace)
   unsigned int* status;
   unsigned long long timeout_ns;
 };
@@ -78,5 +80,18 @@ inline int weight_block(int fmt, int mask) {
   return mask == SHARQ_MASK_PAIR_4_8 ? 32 : 16;
 }
 inline int dense_view_block(int fmt) { return fmt == SHARQ_NVFP4 ? 16 : 32; }
+
+// Split-K plan of the one-CTA kernel: when the output has too few tiles to occupy the SMs,
+// split K so that tiles x splits roughly covers them (each split keeps >= 2 K steps).
+inline int plan_splits(int M, int N, int K, int num_sms) {
+  if (M >= 256 && N % 256 == 0) return 1;  // CTA-pair kernel, enough tiles
+  const int BN = (N % 256 == 0) ? 256 : 128;
+  const int tiles = ((M + 127) / 128) * (N / BN);
+  const int KT = K / 256;
+  if (tiles * 2 > num_sms || KT < 4) return 1;
+  int s = num_sms / tiles;
+  if (s > KT / 2) s = KT / 2;
+  return s < 1 ? 1 : s;
+}
 
 }  // namespace sharq

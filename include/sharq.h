@@ -141,12 +141,24 @@ SHARQ_API sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, c
 SHARQ_API sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* act, void* stream);
 
 /* Y[M x N] = alpha * (sparse-FP4-GEMM(backbone, W) + dense-FP4-GEMM(residual, W)) with
- * alpha = s_g * s_gw, accumulated in one FP32 tensor-memory accumulator and written once
- * (SharQ page, "Core claim": a sparse FP4 GEMM for the backbone and a dense FP4 GEMM
- * for the compensation, sharing one weight payload). Y: device pointer, row-major,
- * y_dtype BF16 (the product) or F32. act->cfg must equal w->cfg and act->K == w->K. */
+ * alpha = s_g * s_gw, accumulated in FP32 tensor memory and written once (SharQ page, "Core
+ * claim": a sparse FP4 GEMM for the backbone and a dense FP4 GEMM for the compensation,
+ * sharing one weight payload). Y: device pointer, row-major, y_dtype BF16 (the product) or
+ * F32. act->cfg must equal w->cfg and act->K == w->K.
+ * workspace / workspace_bytes: optional caller-owned device scratch (16-byte aligned) for
+ * the split-K path used when the output has too few tiles to occupy the GPU (decode-sized
+ * M); sharq_linear_workspace_size gives the bytes it wants. With a NULL or too small
+ * workspace the call runs without splitting K (same result up to summation order, slower
+ * for small M). */
 SHARQ_API sharq_status sharq_linear(const sharq_act* act, const sharq_weight* w, void* Y,
-                          sharq_dtype y_dtype, void* stream);
+                                    sharq_dtype y_dtype, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/* Bytes of workspace sharq_linear uses for this shape on the current device (0 when it does
+ * not split K). Needs the device's SM count: returns SHARQ_ERR_CUDA / SHARQ_ERR_ARCH
+ * without a usable sm_100 device. */
+SHARQ_API sharq_status sharq_linear_workspace_size(int32_t M, int32_t N, int32_t K,
+                                                   sharq_config cfg, size_t* bytes);
 
 /* Synchronises the device, returns and clears the status word the kernels write on a
  * bounded-wait timeout (SHARQ_OK or SHARQ_ERR_TIMEOUT), or SHARQ_ERR_CUDA if the

@@ -103,8 +103,10 @@ def test_null_and_misaligned_pointers_rejected_before_any_launch(sq):
     assert sq.sharq_prepare(p(0x1000), sq.BF16, ctypes.byref(act), None) == 3  # rs misaligned
     w = sq.sharq_weight(p(0x1000), p(0x2000), p(0x3000), p(0x4000), 256, 128, cfg)
     act = sq.sharq_act(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), p(0x6000), 16, 512, cfg)
-    assert sq.sharq_linear(ctypes.byref(act), ctypes.byref(w), p(0x7000), sq.BF16, None) == 1  # K mismatch
-    assert sq.sharq_linear(ctypes.byref(act), ctypes.byref(w), p(0x7000), sq.F16, None) == 1   # bad out dtype
+    assert sq.sharq_linear(ctypes.byref(act), ctypes.byref(w), p(0x7000), sq.BF16, None, 0,
+                           None) == 1  # K mismatch
+    assert sq.sharq_linear(ctypes.byref(act), ctypes.byref(w), p(0x7000), sq.F16, None, 0,
+                           None) == 1  # bad out dtype
 
 
 def test_no_cpu_fallback_without_gpu(sq):
@@ -117,3 +119,12 @@ def test_no_cpu_fallback_without_gpu(sq):
     cfg = sq.Config().c()
     act = sq.sharq_act(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), p(0x6000), 16, 256, cfg)
     assert sq.sharq_prepare(p(0x1000), sq.BF16, ctypes.byref(act), None) in (4, 6)
+
+
+def test_workspace_query_needs_a_device(sq):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    n = ctypes.c_size_t(123)
+    assert sq.sharq_linear_workspace_size(1, 4096, 14336, sq.Config().c(), ctypes.byref(n)) in (4, 6)
+    assert sq.sharq_linear_workspace_size(1, 4096, 14336, sq.Config().c(), None) == 1

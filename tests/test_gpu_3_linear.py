@@ -150,3 +150,33 @@ def test_full_size_sampled_outputs(name, M, K, N, per_row):
     qw = S.quantize_weight(w.values[:, cols], amax=S.amax_of(w.values))
     y64 = S.linear(p, qw)
     check_y(y[np.ix_(rows, cols)], y64, True)
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 14336, 4096), (8, 14336, 4096), (16, 4096, 1024),
+                                   (64, 14336, 4096), (100, 2048, 384)])
+def test_split_k_decode(M, K, N):
+    """Decode-sized M: the split-K path (caller workspace, fixed-order reduction) agrees with
+    the oracle and with the unsplit path, and repeats bit-identically."""
+    import fp4_sparse_dense_b200 as sq
+    import torch
+    rng = np.random.default_rng(M * 31 + N)
+    x = heavy_activations(rng, M, K, per_row=True)
+    w = gaussian_weight(rng, K, N)
+    cfg = cfg_of("nvfp4", "pair48")
+    act = sq.prepare(to_device(x), cfg)
+    wt = sq.quantize_weight(to_device(w), cfg)
+    ws = sq.linear_workspace(M, N, K, cfg)
+    assert ws is not None and ws.numel() >= M * N * 4 * 2
+    y_split = sq.linear(act, wt, out_dtype=torch.float32, workspace=ws)
+    y_split2 = sq.linear(act, wt, out_dtype=torch.float32, workspace=ws)
+    y_plain = sq.linear(act, wt, out_dtype=torch.float32, workspace=None)
+    y_bf16 = sq.linear(act, wt, workspace=ws)
+    torch.cuda.synchronize()
+    assert sq.sharq_device_status() == 0
+    assert torch.equal(y_split, y_split2)
+    p = S.prepare(x.values)
+    qw = S.quantize_weight(w.values)
+    y64 = S.linear(p, qw)
+    check_y(y_split.cpu().numpy().astype(np.float64), y64, False)
+    check_y(y_plain.cpu().numpy().astype(np.float64), y64, False)
+    check_y(y_bf16.float().cpu().numpy().astype(np.float64), y64, True)
