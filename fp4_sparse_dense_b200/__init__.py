@@ -20,12 +20,13 @@ from ._abi import (  # noqa: F401
     sharq_act, sharq_act_bytes, sharq_config, sharq_weight, sharq_weight_bytes, check,
     sharq_act_sizes, sharq_weight_sizes, sharq_status_string, sharq_device_status,
     sharq_prepare, sharq_quantize_weight, sharq_linear, sharq_linear_workspace_size,
+    sharq_linear_noalloc,
 )
 
 __all__ = [
     "Config", "QuantWeight", "PreparedAct", "quantize_weight", "prepare", "linear",
     "sharq_act_sizes", "sharq_weight_sizes", "sharq_prepare", "sharq_quantize_weight",
-    "sharq_linear", "sharq_linear_workspace_size", "sharq_device_status",
+    "sharq_linear", "sharq_linear_workspace_size", "sharq_linear_noalloc", "sharq_device_status",
     "sharq_status_string", "SharqError", "linear_workspace",
     "NVFP4", "MXFP4", "PAIR_4_8", "ELEM_2_4", "F16", "BF16", "F32",
 ]

@@ -65,6 +65,8 @@ def _load():
                               ctypes.c_int, vp, ctypes.c_size_t, vp]),
         "sharq_linear_workspace_size": (st, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                              sharq_config, ctypes.POINTER(ctypes.c_size_t)]),
+        "sharq_linear_noalloc": (st, [ctypes.POINTER(sharq_act), ctypes.POINTER(sharq_weight),
+                                      vp, ctypes.c_int, vp]),
         "sharq_device_status": (st, []),
         "sharq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
@@ -82,6 +84,7 @@ sharq_quantize_weight = lib.sharq_quantize_weight
 sharq_prepare = lib.sharq_prepare
 sharq_linear = lib.sharq_linear
 sharq_linear_workspace_size = lib.sharq_linear_workspace_size
+sharq_linear_noalloc = lib.sharq_linear_noalloc
 sharq_device_status = lib.sharq_device_status
 sharq_status_string = lib.sharq_status_string
 

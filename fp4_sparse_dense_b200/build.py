@@ -14,8 +14,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libsharq.so")
-SOURCES = ["sharq_api.cu", "prep.cu", "quant_weight.cu", "gemm.cu", "gemm_pair.cu"]
-HEADERS = ["fp4_device.cuh", "fp4_quant.cuh", "sm100_ptx.cuh", "sharq_internal.h"]
+SOURCES = ["sharq_api.cu", "prep.cu", "quant_weight.cu", "gemm.cu", "gemm_pair.cu",
+           "noalloc.cu"]
+HEADERS = ["fp4_device.cuh", "fp4_quant.cuh", "sm100_ptx.cuh", "sharq_internal.h",
+           "epilogue.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -160,6 +160,26 @@ SHARQ_API sharq_status sharq_linear(const sharq_act* act, const sharq_weight* w,
 SHARQ_API sharq_status sharq_linear_workspace_size(int32_t M, int32_t N, int32_t K,
                                                    sharq_config cfg, size_t* bytes);
 
+/* sharq_linear for callers that cannot allocate device memory (the SharQ page has no
+ * counterpart: this is a deployment aid, not part of the method). Some callers cannot pass
+ * a workspace: code that runs inside a CUDA graph or an allocator-free runtime, or a host
+ * whose memory manager forbids allocation on the hot path. For decode-sized M, the linear
+ * layer splits K and sums FP32 partials in scratch memory; here that scratch is a fixed
+ * device array compiled into the library, 16 MiB per GPU, held by every GPU that loads
+ * the library until the process exits. The call itself allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine).
+ * - Arguments and result are those of sharq_linear without the workspace; shapes that
+ *   sharq_linear does not split run exactly as sharq_linear with no workspace.
+ * - A shape whose split-K scratch would exceed 16 MiB returns SHARQ_ERR_UNSUPPORTED
+ *   (use sharq_linear with a workspace of sharq_linear_workspace_size bytes instead).
+ * - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *   with that device current); make that first call before any stream capture.
+ * - Every call uses the same array and leaves its partial sums there; nothing in it has to
+ *   start at zero (each call overwrites every value it reads). Calls that overlap on the
+ *   GPU (different streams, or different host threads) race on the array. */
+SHARQ_API sharq_status sharq_linear_noalloc(const sharq_act* act, const sharq_weight* w, void* Y,
+                                            sharq_dtype y_dtype, void* stream);
+
 /* Synchronises the device, returns and clears the status word the kernels write on a
  * bounded-wait timeout (SHARQ_OK or SHARQ_ERR_TIMEOUT), or SHARQ_ERR_CUDA if the
  * synchronisation itself fails. */
