@@ -57,7 +57,14 @@ def src_hash(files):
     return h.hexdigest()[:12]
 
 
-GEMM_SRC = ["fp4_sparse_dense_b200/csrc/gemm.cu", "fp4_sparse_dense_b200/csrc/sm100_ptx.cuh"]
+GEMM_SRC = ["fp4_sparse_dense_b200/csrc/gemm.cu", "fp4_sparse_dense_b200/csrc/gemm_pair.cu",
+            "fp4_sparse_dense_b200/csrc/epilogue.cuh", "fp4_sparse_dense_b200/csrc/sm100_ptx.cuh",
+            "fp4_sparse_dense_b200/csrc/sharq_internal.h"]
+
+
+def gemm_kernel_name(M: int, N: int) -> str:
+    """Which GEMM kernel sharq_linear launches for this shape (CTA pair for M >= 256)."""
+    return "sharq_gemm_pair_kernel" if M >= 256 and N % 256 == 0 else "sharq_gemm_kernel"
 
 
 def traffic_from_profile(workload: str):
@@ -309,7 +316,7 @@ def run_gpu(args):
                          "peak_source": f"{peak_src}: bf16 sustained {bf16_sus} x "
                                         f"{FP4_OVER_BF16} (nominal FP4:BF16)",
                          "ceiling_frac": 2.0 / 3.0,
-                         "kernel": "sharq_gemm_kernel", "kernel_ms": gemm_avg},
+                         "kernel": gemm_kernel_name(M, N), "kernel_ms": gemm_avg},
             "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
                      "frac": prep_gbs / hbm,
                      "bytes_per_elem": PREP_BYTES_PER_ELEM["pair48"],
