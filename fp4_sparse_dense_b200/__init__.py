@@ -125,7 +125,7 @@ def empty_act(M: int, K: int, cfg: Config, device="cuda") -> PreparedAct:
     return PreparedAct(_u8(sz.bq, device), _u8(sz.bs, device), _u8(sz.bm, device),
                        _u8(sz.rq, device) if sz.rq else None,
                        _u8(sz.rs, device) if sz.rs else None,
-                       torch.zeros(4, dtype=torch.float32, device=device), M, K, cfg)
+                       torch.zeros(8, dtype=torch.float32, device=device), M, K, cfg)
 
 
 def quantize_weight(W, cfg: Config = Config(), out: QuantWeight | None = None,

@@ -49,18 +49,17 @@ __device__ __forceinline__ uint32_t quant_nv(const float* v, float s_g, float k,
   if (WANT_DEQ) {
     // E2M1(q) * E4M3(sf) is exact in f16 (at most 6 significant bits, magnitude in
     // [2^-10, 2688]); one float32 rounding for the tensor scale.
+    // scalar __fmul_rn: never merged into a multiply-add with the caller's x - deq
     const __half2 sf2 = __float2half2_rn(sf_val);
-    const float2 sg2 = make_float2(s_g, s_g);
 #pragma unroll
     for (int w = 0; w < N / 8; ++w) {
       uint32_t h[4];
       e2m1x8_to_f16x2(packed[w], h);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float2 f =
-            mul2_rn(__half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[j]), sf2)), sg2);
-        deq[8 * w + 2 * j] = f.x;
-        deq[8 * w + 2 * j + 1] = f.y;
+        const float2 f = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[j]), sf2));
+        deq[8 * w + 2 * j] = __fmul_rn(f.x, s_g);
+        deq[8 * w + 2 * j + 1] = __fmul_rn(f.y, s_g);
       }
     }
   }
@@ -125,6 +124,99 @@ __device__ __forceinline__ uint32_t quant_block(const float* v, TensorConsts c, 
                                                 float* deq) {
   if (FMT == SHARQ_NVFP4) return quant_nv<N, WANT_DEQ>(v, c.s_g, c.k, packed, deq);
   return quant_mx<N, WANT_DEQ>(v, packed, deq);
+}
+
+// One block's scale, split from the per-element work so that a kernel can encode values
+// of one block in any order: `code` is the scale byte (E4M3 or E8M0), `mul` maps a value
+// onto the E2M1 grid (1/d for NVFP4, 2^-e for MXFP4), `sf` is what dequantisation
+// multiplies the E2M1 value by (E4M3(sf) for NVFP4, 2^e for MXFP4), and a block that is
+// not `live` encodes every value as code 0. Same arithmetic as quant_nv / quant_mx.
+struct BlockScale {
+  uint32_t code;
+  float mul;
+  float sf;
+  bool live;
+};
+
+template <int FMT>
+__device__ __forceinline__ BlockScale block_scale(float a, TensorConsts c) {
+  BlockScale b;
+  if (FMT == SHARQ_NVFP4) {
+    b.code = 0;
+    b.sf = 0.f;
+    b.mul = 0.f;
+    b.live = false;
+    if (c.s_g > 0.f) {
+      b.code = cvt_e4m3(__fmul_rn(a, c.k));
+      b.sf = e4m3_value(b.code);
+      const float d = __fmul_rn(b.sf, c.s_g);
+      b.live = d > 0.f;
+      b.mul = b.live ? __frcp_rn(d) : 0.f;
+    }
+  } else {
+    int e = int((__float_as_uint(a) >> 23) & 0xFFu) - 127 - 2;
+    e = max(e, -127);
+    b.live = a > 0.f;
+    if (!b.live) e = -127;
+    b.mul = __uint_as_float(uint32_t(127 - e) << 23);
+    b.sf = pow2f(e);
+    b.code = uint32_t(e + 127);
+  }
+  return b;
+}
+
+// 8 values -> 8 E2M1 codes (v[0] in bits 0..3) with a block's multiplier.
+__device__ __forceinline__ uint32_t encode8(const float* v, const BlockScale& b) {
+  const float2 m2 = make_float2(b.mul, b.mul);
+  const float2 p0 = mul2_rn(make_float2(v[0], v[1]), m2);
+  const float2 p1 = mul2_rn(make_float2(v[2], v[3]), m2);
+  const float2 p2 = mul2_rn(make_float2(v[4], v[5]), m2);
+  const float2 p3 = mul2_rn(make_float2(v[6], v[7]), m2);
+  const uint32_t c = cvt_e2m1x8(p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y);
+  return b.live ? c : 0u;
+}
+
+// 8 E2M1 codes -> their dequantised values: NVFP4 (E2M1 * E4M3(sf)) * s_g, the first
+// product exact in f16; MXFP4 E2M1 * 2^e.
+template <int FMT>
+__device__ __forceinline__ void decode8(uint32_t codes, const BlockScale& b, float s_g,
+                                        float* out) {
+  uint32_t h[4];
+  e2m1x8_to_f16x2(codes, h);
+  if (FMT == SHARQ_NVFP4) {
+    // The s_g product uses the scalar __fmul_rn, which is never merged into a multiply-add:
+    // ptxas contracts the packed mul.rn.f32x2 with a following sub.rn.f32x2 (r = x - deq)
+    // into one fused operation, which skips this rounding.
+    const __half2 sf2 = __float2half2_rn(b.sf);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[j]), sf2));
+      out[2 * j] = __fmul_rn(f.x, s_g);
+      out[2 * j + 1] = __fmul_rn(f.y, s_g);
+    }
+  } else {
+    // E2M1 * 2^e is exact, so a fused x - deq downstream cannot change the result
+    const float2 p2 = make_float2(b.sf, b.sf);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = mul2_rn(__half22float2(*reinterpret_cast<const __half2*>(&h[j])), p2);
+      out[2 * j] = f.x;
+      out[2 * j + 1] = f.y;
+    }
+  }
+}
+
+// max |v| over N values (N a multiple of 2) with the three-input max of sm_100.
+template <int N>
+__device__ __forceinline__ float amax_n(const float* v) {
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < N; i += 2) {
+    float t;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(t) : "f"(a), "f"(v[i]), "f"(v[i + 1]));
+    a = t;
+  }
+  return a;
 }
 
 // byte offset of (row r, column c) inside a staged tile of 128 rows x C scale columns

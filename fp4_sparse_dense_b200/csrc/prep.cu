@@ -19,6 +19,7 @@
 #include "fp4_device.cuh"
 #include "fp4_quant.cuh"
 #include "sharq_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace sharq {
 
@@ -61,9 +62,11 @@ __global__ void __launch_bounds__(512) amax_kernel(const uint4* __restrict__ X, 
 
 // Entry of the top-2-of-4 decision table. Bit b of `idx` is one comparison "candidate i
 // beats candidate j" (i < j; a tie is won by i) in the order (0,1) (0,2) (0,3) (1,2)
-// (1,3) (2,3). A candidate is kept when fewer than two others beat it; the entry is the
-// metadata nibble i0 | i1 << 2 of the two kept candidates (i0 < i1).
-__device__ __forceinline__ uint8_t top2_entry(int idx) {
+// (1,3) (2,3). A candidate is kept when fewer than two others beat it. The entry packs
+//   bits  0..15  byte selector that keeps the kept pairs' code bytes and zeroes the others
+//   bits 16..23  byte selector of the two kept bytes (i0, i1) in order
+//   bits 24..27  metadata nibble i0 | i1 << 2 (i0 < i1)
+__device__ __forceinline__ uint32_t top2_entry(int idx) {
   const int c01 = idx & 1, c02 = (idx >> 1) & 1, c03 = (idx >> 2) & 1;
   const int c12 = (idx >> 3) & 1, c13 = (idx >> 4) & 1, c23 = (idx >> 5) & 1;
   const int rank[4] = {3 - c01 - c02 - c03, c01 + 2 - c12 - c13, c02 + c12 + 1 - c23,
@@ -74,23 +77,97 @@ __device__ __forceinline__ uint8_t top2_entry(int idx) {
       if (i0 < 0) i0 = j;
       else if (i1 < 0) i1 = j;
     }
-  if (i0 < 0 || i1 < 0) return 0x4;  // not reachable from a total order
-  return uint8_t(i0 | (i1 << 2));
-}
-
-// Ranking key of a pair (two 16-bit inputs in one word): the larger 15-bit magnitude in
-// the high half, the smaller in the low half. For bf16 and fp16 the magnitude order of
-// the values is the unsigned order of these bit fields.
-__device__ __forceinline__ uint32_t pair_key(uint32_t w) {
-  const uint32_t m = w & 0x7FFF7FFFu;
-  const uint32_t sw = __byte_perm(m, 0, 0x1032);
-  return __byte_perm(__vmaxu2(m, sw), __vminu2(m, sw), 0x3254);
+  if (i0 < 0 || i1 < 0) {  // not reachable from a total order
+    i0 = 0;
+    i1 = 1;
+  }
+  uint32_t keep = 0;
+  for (int j = 0; j < 4; ++j) keep |= uint32_t(j == i0 || j == i1 ? j : 4) << (4 * j);
+  return keep | (uint32_t(i0 | (i1 << 4)) << 16) | (uint32_t(i0 | (i1 << 2)) << 24);
 }
 
 template <bool BF16>
-__device__ __forceinline__ float lo16(uint32_t w) { return in_to_float<BF16>(w & 0xFFFFu); }
+__device__ __forceinline__ float lo16(uint32_t w) {
+  return BF16 ? __uint_as_float(w << 16) : in_to_float<false>(w & 0xFFFFu);
+}
 template <bool BF16>
-__device__ __forceinline__ float hi16(uint32_t w) { return in_to_float<BF16>(w >> 16); }
+__device__ __forceinline__ float hi16(uint32_t w) {
+  return BF16 ? __uint_as_float(w & 0xFFFF0000u) : in_to_float<false>(w >> 16);
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Tensor amax inside the preparation launch. Every CTA folds its share of X into
+// acc[gen & 1] with atomicMax, then waits at a grid barrier (all CTAs are resident: the
+// kernel is launched cooperatively). The barrier's last arrival resets `count` and
+// advances `gen`; CTA 0 clears the other accumulator for the next call. The state lives in
+// words 2..5 of the caller's tensor-scale buffer, which start at zero.
+struct AmaxState {
+  unsigned acc[2];
+  unsigned count;
+  unsigned gen;
+};
+
+template <bool BF16>
+__device__ float grid_amax(const uint4* __restrict__ X, size_t n16, AmaxState* st,
+                           unsigned* status, uint64_t limit_ns, bool* ok) {
+  __shared__ unsigned s_gen, s_red[8], s_ok;
+  if (threadIdx.x == 0) s_gen = ld_acquire_gpu(&st->gen);
+  uint32_t m = 0;
+  const size_t stride = size_t(gridDim.x) * blockDim.x;
+#pragma unroll 1
+  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n16; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      v[j] = i + j * stride < n16 ? __ldg(X + i + j * stride) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      m = __vmaxu2(m, v[j].x & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v[j].y & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v[j].z & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v[j].w & 0x7FFF7FFFu);
+    }
+  }
+  uint32_t h = max(m & 0xFFFFu, m >> 16);
+  for (int off = 16; off; off >>= 1) h = max(h, __shfl_xor_sync(0xFFFFFFFFu, h, off));
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = h;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0;
+    for (int i = 0; i < int(blockDim.x >> 5); ++i) b = max(b, s_red[i]);
+    const unsigned gen = s_gen;
+    atomicMax(&st->acc[gen & 1u], __float_as_uint(in_to_float<BF16>(b)));
+    __threadfence();
+    unsigned good = 1;
+    if (atomicAdd(&st->count, 1u) == gridDim.x - 1) {
+      st->count = 0;
+      __threadfence();
+      atomicAdd(&st->gen, 1u);
+    } else {
+      const uint64_t t0 = ptx::globaltimer();
+      for (uint32_t it = 1; ld_acquire_gpu(&st->gen) == gen; ++it) {
+        if ((it & 255u) == 0 && ptx::globaltimer() - t0 > limit_ns) {
+          atomicExch(status, unsigned(SHARQ_ERR_TIMEOUT));
+          good = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    s_red[0] = good ? ld_acquire_gpu(&st->acc[gen & 1u]) : 0u;
+    s_ok = good;
+    if (blockIdx.x == 0) st->acc[(gen + 1u) & 1u] = 0u;
+  }
+  __syncthreads();
+  *ok = s_ok != 0;
+  return __uint_as_float(s_red[0]);
+}
 
 // Pair-wise 4:8 mask: in every 8 consecutive K keep the 2 of the 4 adjacent pairs with the
 // largest (max |x|, min |x|), ties to the lower pair; the kept values (compressed, 16 per
@@ -100,51 +177,71 @@ __device__ __forceinline__ float hi16(uint32_t w) { return in_to_float<BF16>(w >
 // unit = 32 K); warps walk the items with a grid stride, loading the next item while
 // computing the current one. Scale and metadata bytes of neighbouring lanes are gathered
 // with shuffles into 32-bit stores, so no CTA barrier is needed inside the loop.
+//
+// Per unit the backbone is encoded at all 32 positions with the block's scale (its max
+// |x| is the unit's max |x|: the largest element of every group of 8 lies in its top pair,
+// which is kept); byte permutes then keep the kept pairs' code bytes, either compressed
+// (the backbone operand) or in place with zeros elsewhere, which dequantise to the backbone
+// at kept positions and +0 elsewhere, so r = x - deq needs no per-element selection.
 template <bool BF16, int FMT, bool RESIDUAL>
 __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   constexpr int RB = FMT == SHARQ_NVFP4 ? 16 : 32;  // residual block
-  __shared__ uint8_t s_top2[64];
+  __shared__ uint32_t s_top2[64];
   if (threadIdx.x < 64) s_top2[threadIdx.x] = top2_entry(threadIdx.x);
 
   TensorConsts tc{1.f, 1.f};
   if (FMT == SHARQ_NVFP4) {
-    tc = tensor_consts(__uint_as_float(*reinterpret_cast<const unsigned int*>(p.amax)));
-    if (blockIdx.x == 0 && threadIdx.x == 0) *p.tensor_scale = tc.s_g;
+    bool ok = true;
+    const float amax = grid_amax<BF16>(static_cast<const uint4*>(p.X),
+                                       size_t(p.M) * size_t(p.K) / 8,
+                                       reinterpret_cast<AmaxState*>(p.tensor_scale + 2),
+                                       p.status, p.timeout_ns, &ok);
+    if (!ok) return;
+    tc = tensor_consts(amax);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      p.tensor_scale[0] = tc.s_g;
+      p.tensor_scale[1] = amax;
+    }
   } else if (blockIdx.x == 0 && threadIdx.x == 0) {
-    *p.tensor_scale = 1.0f;
+    p.tensor_scale[0] = 1.0f;
   }
   __syncthreads();  // decision table ready
 
   const int K = p.K, M = p.M, Mp = p.Mp;
-  const int KS = K / 256;                   // 256-K slices
+  const int KS = K / 256;  // 256-K slices
   const int n_items = (Mp / 4) * KS;
   const int lane = threadIdx.x & 31;
-  const int u = lane & 7;                   // 32-K unit inside the slice
-  const int rsub = lane >> 3;               // row inside the item
+  const int u = lane & 7;    // 32-K unit inside the slice
+  const int rsub = lane >> 3;  // row inside the item
   const int stride = gridDim.x * (blockDim.x >> 5);
+  const int stride_q = stride % KS, stride_r = (stride / KS) * 4;
   const uint16_t* X = static_cast<const uint16_t*>(p.X);
   const size_t scols_b = size_t(K) / 32 / 4;  // 512-byte chunks per 128 rows (backbone)
   const size_t scols_r = size_t(K) / RB / 4;  // (residual)
 
   int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int q = item % KS;                // slice of the current item
+  int row = (item / KS) * 4 + rsub;  // row of this lane in the current item
   uint4 cur[4];
-  auto load = [&](int it, uint4* dst) {
-    const int row = (it / KS) * 4 + rsub;
-    if (it < n_items && row < M) {
+  auto load = [&](int it, int r, int qq, uint4* dst) {
+    if (it < n_items && r < M) {
       const uint4* src =
-          reinterpret_cast<const uint4*>(X + size_t(row) * K + size_t(it % KS) * 256 + u * 32);
+          reinterpret_cast<const uint4*>(X + size_t(r) * K + size_t(qq) * 256 + u * 32);
 #pragma unroll
       for (int i = 0; i < 4; ++i) dst[i] = __ldg(src + i);
     }
   };
-  load(item, cur);
+  load(item, row, q, cur);
 
 #pragma unroll 1
   for (; item < n_items; item += stride) {
+    int nq = q + stride_q, nrow = row + stride_r;
+    if (nq >= KS) {
+      nq -= KS;
+      nrow += 4;
+    }
     uint4 nxt[4];
-    load(item + stride, nxt);
-    const int q = item % KS;
-    const int row = (item / KS) * 4 + rsub;
+    load(item + stride, nrow, nq, nxt);
     const int k0 = q * 256 + u * 32;
     const bool live = row < M;
     uint32_t w[16];
@@ -156,65 +253,72 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
 
     uint32_t meta = 0x4444u, bsf = 0, rsf0 = 0, rsf1 = 0;
     if (live) {
-      // ---- mask: one table lookup per group of 4 pairs
-      int sel0[4], sel1[4];
-      float comp[16];
-      meta = 0;
+      // ---- mask: pair keys (max |x| << 16 | min |x|, as 15-bit magnitudes) and one
+      // table entry per group of 4 pairs; the comparison bits are the sign bits of
+      // key_j - key_i - 1, shifted in from (2,3) down to (0,1)
+      uint32_t L[4];
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        const uint32_t ka = pair_key(w[4 * g]), kb = pair_key(w[4 * g + 1]);
-        const uint32_t kc = pair_key(w[4 * g + 2]), kd = pair_key(w[4 * g + 3]);
-        const int idx = int(ka >= kb) | (int(ka >= kc) << 1) | (int(ka >= kd) << 2) |
-                        (int(kb >= kc) << 3) | (int(kb >= kd) << 4) | (int(kc >= kd) << 5);
-        const uint32_t nib = s_top2[idx];
-        const int i0 = int(nib & 3u), i1 = int(nib >> 2);
-        sel0[g] = i0;
-        sel1[g] = i1;
-        meta |= nib << (4 * g);
-        const uint32_t a = i0 == 0 ? w[4 * g] : (i0 == 1 ? w[4 * g + 1] : w[4 * g + 2]);
-        const uint32_t b = i1 == 3 ? w[4 * g + 3] : (i1 == 2 ? w[4 * g + 2] : w[4 * g + 1]);
-        comp[4 * g + 0] = lo16<BF16>(a);
-        comp[4 * g + 1] = hi16<BF16>(a);
-        comp[4 * g + 2] = lo16<BF16>(b);
-        comp[4 * g + 3] = hi16<BF16>(b);
+        uint32_t k[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t m = w[4 * g + j] & 0x7FFF7FFFu;
+          k[j] = max(m, __byte_perm(m, 0, 0x1032));
+        }
+        uint32_t idx = (k[3] - k[2] - 1u) >> 31;
+        idx = __funnelshift_l(k[3] - k[1] - 1u, idx, 1);
+        idx = __funnelshift_l(k[2] - k[1] - 1u, idx, 1);
+        idx = __funnelshift_l(k[3] - k[0] - 1u, idx, 1);
+        idx = __funnelshift_l(k[2] - k[0] - 1u, idx, 1);
+        idx = __funnelshift_l(k[1] - k[0] - 1u, idx, 1);
+        L[g] = s_top2[idx];
       }
-      // ---- backbone: one block of the 16 kept values
-      uint32_t bcodes[2];
-      float deq[16];
-      bsf = quant_block<FMT, 16, RESIDUAL>(comp, tc, bcodes, deq);
+      meta = ((L[0] >> 24) & 0xFu) | ((L[1] >> 20) & 0xF0u) | ((L[2] >> 16) & 0xF00u) |
+             ((L[3] >> 12) & 0xF000u);
+
+      float x[32];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        x[2 * i] = lo16<BF16>(w[i]);
+        x[2 * i + 1] = hi16<BF16>(w[i]);
+      }
+      // ---- backbone: one block of 32 logical K
+      const BlockScale bb = block_scale<FMT>(amax_n<32>(x), tc);
+      bsf = bb.code;
+      uint32_t c[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) c[g] = encode8(x + 8 * g, bb);
+      // compressed backbone codes: the kept bytes of groups 0, 1 and of groups 2, 3 (the
+      // selector takes bytes i0, i1 of the first word and 4 + i0, 4 + i1 of the second)
+      const uint32_t sel01 = __byte_perm(L[0], L[1], 0x0062u) + 0x4400u;
+      const uint32_t sel23 = __byte_perm(L[2], L[3], 0x0062u) + 0x4400u;
       *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.bq) + size_t(row) * (K / 4) + k0 / 4) =
-          make_uint2(bcodes[0], bcodes[1]);
+          make_uint2(__byte_perm(c[0], c[1], sel01), __byte_perm(c[2], c[3], sel23));
       if (RESIDUAL) {
-        // ---- residual against the quantised backbone: r = x - deq on kept pairs and
-        // x - 0 == x (exactly, -0 included) elsewhere; quantised per residual block
+        // ---- residual against the quantised backbone
+        float r[32];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float d[8];
+          decode8<FMT>(__byte_perm(c[g], 0u, L[g]), bb, tc.s_g, d);
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            const float2 t = sub2_rn(make_float2(x[8 * g + j], x[8 * g + j + 1]),
+                                     make_float2(d[j], d[j + 1]));
+            r[8 * g + j] = t.x;
+            r[8 * g + j + 1] = t.y;
+          }
+        }
+        uint32_t rc[4];
 #pragma unroll
         for (int hb = 0; hb < 32 / RB; ++hb) {
-          constexpr int G = RB / 8;  // groups per residual block
-          float rv[RB];
+          const BlockScale rb = block_scale<FMT>(amax_n<RB>(r + hb * RB), tc);
+          if (hb == 0) rsf0 = rb.code; else rsf1 = rb.code;
 #pragma unroll
-          for (int gg = 0; gg < G; ++gg) {
-            const int g = hb * G + gg;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t wj = w[4 * g + j];
-              const bool f0 = sel0[g] == j, f1 = sel1[g] == j;
-              const float2 d = make_float2(f0 ? deq[4 * g] : (f1 ? deq[4 * g + 2] : 0.f),
-                                           f0 ? deq[4 * g + 1] : (f1 ? deq[4 * g + 3] : 0.f));
-              const float2 r = sub2_rn(make_float2(lo16<BF16>(wj), hi16<BF16>(wj)), d);
-              rv[8 * gg + 2 * j] = r.x;
-              rv[8 * gg + 2 * j + 1] = r.y;
-            }
-          }
-          uint32_t rcodes[RB / 8];
-          const uint32_t sfr = quant_block<FMT, RB, false>(rv, tc, rcodes, nullptr);
-          if (hb == 0) rsf0 = sfr; else rsf1 = sfr;
-          uint8_t* dst =
-              static_cast<uint8_t*>(p.rq) + size_t(row) * (K / 2) + k0 / 2 + hb * (RB / 2);
-          if constexpr (RB == 16)
-            *reinterpret_cast<uint2*>(dst) = make_uint2(rcodes[0], rcodes[1]);
-          else
-            *reinterpret_cast<uint4*>(dst) = make_uint4(rcodes[0], rcodes[1], rcodes[2], rcodes[3]);
+          for (int g = 0; g < RB / 8; ++g) rc[hb * (RB / 8) + g] = encode8(r + hb * RB + 8 * g, rb);
         }
+        *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.rq) + size_t(row) * (K / 2) + k0 / 2) =
+            make_uint4(rc[0], rc[1], rc[2], rc[3]);
       }
     }
 
@@ -261,6 +365,8 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+    q = nq;
+    row = nrow;
   }
 }
 
@@ -419,13 +525,23 @@ template <bool BF16, int FMT, bool RES>
 static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
   if (mask == SHARQ_MASK_PAIR_4_8) {
     auto kern = prep_pair_kernel<BF16, FMT, RES>;
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
-    if (e != cudaSuccess) return e;
+    static int per_sm = 0;  // resident CTAs per SM (one value per instantiation)
+    if (per_sm == 0) {
+      cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+      if (e != cudaSuccess) return e;
+      if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    }
     const long items = long(p.Mp / 4) * (p.K / 256);
     long blocks = (items + 7) / 8;
-    const long cap = long(num_sms) * (per_sm > 0 ? per_sm : 1);
+    const long cap = long(num_sms) * per_sm;
     if (blocks > cap) blocks = cap;
+    if (FMT == SHARQ_NVFP4) {
+      // the in-kernel tensor amax waits for every CTA: launch them all resident
+      PrepParams q = p;
+      void* args[] = {&q};
+      return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(unsigned(blocks)),
+                                         dim3(256), args, 0, st);
+    }
     kern<<<unsigned(blocks), 256, 0, st>>>(p);
   } else {
     dim3 grid(p.K / 256, (p.M + 127) / 128);

@@ -293,7 +293,9 @@ sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* a,
   if ((s = device_info(&d)) != SHARQ_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == SHARQ_BF16;
-  if (a->cfg.fmt == SHARQ_NVFP4) {
+  // the pair-mask kernel reduces the NVFP4 tensor amax itself (state in tensor_scale[2..5]);
+  // the element-mask kernel takes it from a separate pass into tensor_scale[1]
+  if (a->cfg.fmt == SHARQ_NVFP4 && a->cfg.mask == SHARQ_MASK_ELEM_2_4) {
     if (cudaMemsetAsync(a->tensor_scale + 1, 0, sizeof(float), st) != cudaSuccess)
       return SHARQ_ERR_CUDA;
     s = from_cuda(launch_amax(X, bf16, size_t(a->M) * size_t(a->K),
@@ -312,6 +314,8 @@ sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* a,
   p.M = a->M;
   p.K = a->K;
   p.Mp = int(round_up(size_t(a->M), 128));
+  p.status = d.status;
+  p.timeout_ns = kWaitLimitNs;
   return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
 }
 

@@ -16,9 +16,11 @@ struct PrepParams {
   void* bm;
   void* rq;
   void* rs;
-  float* tensor_scale;  // [0] = s_g (written), [1] = amax (NVFP4, read)
-  const float* amax;    // = tensor_scale + 1
+  float* tensor_scale;  // [0] = s_g, [1] = amax (written); [2..5] amax state (pair mask, NVFP4)
+  const float* amax;    // = tensor_scale + 1 (element mask, NVFP4: written by amax_kernel)
   int M, K, Mp;
+  unsigned* status;     // device status word (bounded-wait timeouts)
+  unsigned long long timeout_ns;
 };
 
 struct WeightQuantParams {
