@@ -320,14 +320,15 @@ def run_gpu(args):
             "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
                      "frac": prep_gbs / hbm,
                      "bytes_per_elem": PREP_BYTES_PER_ELEM["pair48"],
-                     "kernel": "prep_pair_kernel",
-                     "note": "one launch: tensor amax (first pass over X) + fused preparation; "
-                             "algorithmic bytes count X once"},
+                     "kernel": "prep_mask_kernel + prep_pair_kernel",
+                     "note": "two launches (mask, metadata and tensor amax; then quantisation, "
+                             "started early by programmatic dependent launch); algorithmic "
+                             "bytes count X once"},
             "gemm_tflops": gemm_tflops,
             "pct_fp4_peak": 100.0 * gemm_tflops / fp4_peak,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
                     "d2h_bytes_per_step": M * N * 2},
-            "gpu_launches": (1 + 1 + (1 if WS is not None else 0)) * args.steps,
+            "gpu_launches": (2 + 1 + (1 if WS is not None else 0)) * args.steps,
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline and world == 1:

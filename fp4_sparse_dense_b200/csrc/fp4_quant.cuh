@@ -165,6 +165,49 @@ __device__ __forceinline__ BlockScale block_scale(float a, TensorConsts c) {
   return b;
 }
 
+// NVFP4 block scale from per-tensor tables: for every E4M3 code c (0..127) of one tensor,
+// inv[c] = 1 / (E4M3(c) * s_g) (0 when that product is 0) and sfh[c] = E4M3(c) as an f16
+// pair. Built once per CTA after s_g is known; gives exactly block_scale<SHARQ_NVFP4>.
+struct NvScaleTable {
+  float inv[128];
+  uint32_t sfh[128];
+};
+
+__device__ __forceinline__ void nv_table_fill(NvScaleTable* t, float s_g, int tid) {
+  if (tid < 128) {
+    const float sf = e4m3_value(uint32_t(tid));
+    const float d = __fmul_rn(sf, s_g);
+    t->inv[tid] = d > 0.f ? __frcp_rn(d) : 0.f;
+    const __half2 h = __float2half2_rn(sf);
+    t->sfh[tid] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+}
+
+__device__ __forceinline__ BlockScale nv_block_scale(float a, TensorConsts c,
+                                                     const NvScaleTable* t) {
+  BlockScale b;
+  b.code = cvt_e4m3(__fmul_rn(a, c.k));  // k = 0 for an all-zero tensor: code 0
+  b.mul = t->inv[b.code];
+  b.live = b.mul > 0.f;
+  b.sf = __uint_as_float(t->sfh[b.code]);  // f16 pair bits, read by decode8_nv
+  return b;
+}
+
+// decode8 for a block from nv_block_scale (sf holds the E4M3 value as an f16 pair)
+__device__ __forceinline__ void decode8_nv(uint32_t codes, const BlockScale& b, float s_g,
+                                           float* out) {
+  uint32_t h[4];
+  e2m1x8_to_f16x2(codes, h);
+  const uint32_t sfh = __float_as_uint(b.sf);
+  const __half2 sf2 = *reinterpret_cast<const __half2*>(&sfh);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[j]), sf2));
+    out[2 * j] = __fmul_rn(f.x, s_g);  // never merged into a multiply-add
+    out[2 * j + 1] = __fmul_rn(f.y, s_g);
+  }
+}
+
 // 8 values -> 8 E2M1 codes (v[0] in bits 0..3) with a block's multiplier.
 __device__ __forceinline__ uint32_t encode8(const float* v, const BlockScale& b) {
   const float2 m2 = make_float2(b.mul, b.mul);

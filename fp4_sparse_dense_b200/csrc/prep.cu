@@ -95,44 +95,20 @@ __device__ __forceinline__ float hi16(uint32_t w) {
   return BF16 ? __uint_as_float(w & 0xFFFF0000u) : in_to_float<false>(w >> 16);
 }
 
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Tensor amax inside the preparation launch. Every CTA folds its share of X into
-// acc[gen & 1] with atomicMax, then waits at a grid barrier (all CTAs are resident: the
-// kernel is launched cooperatively). The barrier's last arrival resets `count` and
-// advances `gen`; CTA 0 clears the other accumulator for the next call. The state lives in
-// words 2..5 of the caller's tensor-scale buffer, which start at zero.
+// NVFP4 tensor amax across the two preparation kernels, in words 2..3 of the caller's
+// tensor-scale buffer (zero before the first call): the mask kernel folds max |x| into
+// `acc` with atomicMax; every CTA of the quantisation kernel reads it once and counts
+// itself in `done`, and the CTA that completes the count sets both back to zero for the
+// next call. No CTA waits for another.
 struct AmaxState {
-  unsigned acc[2];
-  unsigned count;
-  unsigned gen;
+  unsigned acc;   // max |x| as float bits (non-negative floats order like their bits)
+  unsigned done;  // CTAs of the quantisation kernel that have read acc
 };
 
+// CTA max of the threads' packed 15-bit magnitudes (two per word), folded into st->acc.
 template <bool BF16>
-__device__ float grid_amax(const uint4* __restrict__ X, size_t n16, AmaxState* st,
-                           unsigned* status, uint64_t limit_ns, bool* ok) {
-  __shared__ unsigned s_gen, s_red[8], s_ok;
-  if (threadIdx.x == 0) s_gen = ld_acquire_gpu(&st->gen);
-  uint32_t m = 0;
-  const size_t stride = size_t(gridDim.x) * blockDim.x;
-#pragma unroll 1
-  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n16; i += 4 * stride) {
-    uint4 v[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      v[j] = i + j * stride < n16 ? __ldg(X + i + j * stride) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      m = __vmaxu2(m, v[j].x & 0x7FFF7FFFu);
-      m = __vmaxu2(m, v[j].y & 0x7FFF7FFFu);
-      m = __vmaxu2(m, v[j].z & 0x7FFF7FFFu);
-      m = __vmaxu2(m, v[j].w & 0x7FFF7FFFu);
-    }
-  }
+__device__ void block_max_to(uint32_t m, AmaxState* st) {
+  __shared__ unsigned s_red[8];
   uint32_t h = max(m & 0xFFFFu, m >> 16);
   for (int off = 16; off; off >>= 1) h = max(h, __shfl_xor_sync(0xFFFFFFFFu, h, off));
   if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = h;
@@ -140,43 +116,157 @@ __device__ float grid_amax(const uint4* __restrict__ X, size_t n16, AmaxState* s
   if (threadIdx.x == 0) {
     uint32_t b = 0;
     for (int i = 0; i < int(blockDim.x >> 5); ++i) b = max(b, s_red[i]);
-    const unsigned gen = s_gen;
-    atomicMax(&st->acc[gen & 1u], __float_as_uint(in_to_float<BF16>(b)));
-    __threadfence();
-    unsigned good = 1;
-    if (atomicAdd(&st->count, 1u) == gridDim.x - 1) {
-      st->count = 0;
-      __threadfence();
-      atomicAdd(&st->gen, 1u);
-    } else {
-      const uint64_t t0 = ptx::globaltimer();
-      for (uint32_t it = 1; ld_acquire_gpu(&st->gen) == gen; ++it) {
-        if ((it & 255u) == 0 && ptx::globaltimer() - t0 > limit_ns) {
-          atomicExch(status, unsigned(SHARQ_ERR_TIMEOUT));
-          good = 0;
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    __threadfence();
-    s_red[0] = good ? ld_acquire_gpu(&st->acc[gen & 1u]) : 0u;
-    s_ok = good;
-    if (blockIdx.x == 0) st->acc[(gen + 1u) & 1u] = 0u;
+    atomicMax(&st->acc, __float_as_uint(in_to_float<BF16>(b)));
   }
+}
+
+// Table entry of a metadata nibble i0 | i1 << 2 (same packing as top2_entry); nibbles that
+// the mask never produces map to pairs (0, 1).
+__device__ __forceinline__ uint32_t nibble_entry(int nib) {
+  int i0 = nib & 3, i1 = nib >> 2;
+  if (!(i0 < i1)) {
+    i0 = 0;
+    i1 = 1;
+  }
+  uint32_t keep = 0;
+  for (int j = 0; j < 4; ++j) keep |= uint32_t(j == i0 || j == i1 ? j : 4) << (4 * j);
+  return keep | (uint32_t(i0 | (i1 << 4)) << 16) | (uint32_t(i0 | (i1 << 2)) << 24);
+}
+
+// Pair-wise 4:8 mask of one 32-K unit (16 words of two 16-bit inputs): one table entry per
+// group of 4 pairs from the pair keys (max |x| << 16 | min |x|, as 15-bit magnitudes); the
+// comparison bits are the sign bits of key_j - key_i - 1, shifted in from (2,3) down to
+// (0,1). Returns the unit's 4 metadata nibbles; folds the magnitudes into *mx.
+__device__ __forceinline__ uint32_t pair_mask(const uint32_t* w, const uint32_t* top2,
+                                              uint32_t* L, uint32_t* mx) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint32_t k[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t m = w[4 * g + j] & 0x7FFF7FFFu;
+      *mx = __vmaxu2(*mx, m);
+      k[j] = max(m, __byte_perm(m, 0, 0x1032));
+    }
+    uint32_t idx = (k[3] - k[2] - 1u) >> 31;
+    idx = __funnelshift_l(k[3] - k[1] - 1u, idx, 1);
+    idx = __funnelshift_l(k[2] - k[1] - 1u, idx, 1);
+    idx = __funnelshift_l(k[3] - k[0] - 1u, idx, 1);
+    idx = __funnelshift_l(k[2] - k[0] - 1u, idx, 1);
+    idx = __funnelshift_l(k[1] - k[0] - 1u, idx, 1);
+    L[g] = top2[idx];
+  }
+  return ((L[0] >> 24) & 0xFu) | ((L[1] >> 20) & 0xF0u) | ((L[2] >> 16) & 0xF00u) |
+         ((L[3] >> 12) & 0xF000u);
+}
+
+// Warp items of the pair-mask kernels: an item is 4 rows x 256 K (lane = row * 8 + unit,
+// unit = 32 K); warps walk the items with a grid stride. Offsets are 32-bit: sharq_prepare
+// admits M * K < 2^31 only.
+struct PairWalk {
+  int K, M, Mp, KS, n_items, u, stride, stride_q, stride_r, first, q0, row0;
+  const uint16_t* X;
+  uint8_t* bm;
+
+  __device__ __forceinline__ PairWalk(const PrepParams& p) {
+    K = p.K;
+    M = p.M;
+    Mp = p.Mp;
+    KS = K / 256;
+    n_items = (Mp / 4) * KS;
+    const int lane = threadIdx.x & 31;
+    u = lane & 7;
+    stride = gridDim.x * (blockDim.x >> 5);
+    stride_q = stride % KS;
+    stride_r = (stride / KS) * 4;
+    first = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    q0 = first % KS;
+    row0 = (first / KS) * 4 + (lane >> 3);
+    X = static_cast<const uint16_t*>(p.X);
+    bm = static_cast<uint8_t*>(p.bm);
+  }
+  __device__ __forceinline__ void load(int it, int r, int q, uint4* dst) const {
+    if (it < n_items && r < M) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          X + (uint32_t(r) * uint32_t(K) + uint32_t(q) * 256u + uint32_t(u) * 32u));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = __ldg(src + i);
+    }
+  }
+  __device__ __forceinline__ void advance(int& q, int& r) const {
+    q += stride_q;
+    r += stride_r;
+    if (q >= KS) {
+      q -= KS;
+      r += 4;
+    }
+  }
+  // metadata: 4 nibbles per lane, the row's 16 bytes at slice q
+  __device__ __forceinline__ uint32_t meta_off(int q, int r) const {
+    return uint32_t(q) * uint32_t(Mp) * 16u + uint32_t(r) * 16u + uint32_t(u) * 2u;
+  }
+  // lanes u, u+1 -> one 32-bit store (whole warp)
+  __device__ __forceinline__ void store_meta(int q, int r, uint32_t meta) const {
+    const uint32_t m16 = meta & 0xFFFFu;
+    const uint32_t word = m16 | (__shfl_down_sync(0xFFFFFFFFu, m16, 1) << 16);
+    if ((u & 1) == 0) *reinterpret_cast<uint32_t*>(bm + meta_off(q, r)) = word;
+  }
+};
+
+__device__ __forceinline__ void unpack16(const uint4* c, uint32_t* w) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    w[4 * i + 0] = c[i].x; w[4 * i + 1] = c[i].y;
+    w[4 * i + 2] = c[i].z; w[4 * i + 3] = c[i].w;
+  }
+}
+
+// First NVFP4 preparation kernel (pair mask): streams X from HBM, computes the mask, writes
+// the metadata (padding rows included) and folds max |x| into the tensor amax. Its integer
+// work hides under the HBM reads.
+template <bool BF16>
+__global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
+  // the quantisation kernel may start its prologue now; it waits for this grid's completion
+  // (griddepcontrol.wait) before it reads anything written here
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ uint32_t s_top2[64];
+  if (threadIdx.x < 64) s_top2[threadIdx.x] = top2_entry(threadIdx.x);
   __syncthreads();
-  *ok = s_ok != 0;
-  return __uint_as_float(s_red[0]);
+  const PairWalk wk(p);
+  uint32_t mx = 0;
+  int q = wk.q0, row = wk.row0;
+  uint4 cur[4];
+  wk.load(wk.first, row, q, cur);
+#pragma unroll 1
+  for (int item = wk.first; item < wk.n_items; item += wk.stride) {
+    int nq = q, nrow = row;
+    wk.advance(nq, nrow);
+    uint4 nxt[4];
+    wk.load(item + wk.stride, nrow, nq, nxt);
+    uint32_t meta = 0x4444u;  // padding rows: pairs 0, 1
+    if (row < wk.M) {
+      uint32_t w[16], L[4];
+      unpack16(cur, w);
+      meta = pair_mask(w, s_top2, L, &mx);
+    }
+    wk.store_meta(q, row, meta);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+    q = nq;
+    row = nrow;
+  }
+  block_max_to<BF16>(mx, reinterpret_cast<AmaxState*>(p.tensor_scale + 2));
 }
 
 // Pair-wise 4:8 mask: in every 8 consecutive K keep the 2 of the 4 adjacent pairs with the
 // largest (max |x|, min |x|), ties to the lower pair; the kept values (compressed, 16 per
 // 32 K) form one backbone block; the residual is taken against their dequantised values.
 //
-// Persistent and warp-independent: a warp item is 4 rows x 256 K (lane = row * 8 + unit,
-// unit = 32 K); warps walk the items with a grid stride, loading the next item while
-// computing the current one. Scale and metadata bytes of neighbouring lanes are gathered
-// with shuffles into 32-bit stores, so no CTA barrier is needed inside the loop.
+// Persistent and warp-independent (PairWalk), loading the next item while computing the
+// current one. Scale and metadata bytes of neighbouring lanes are gathered with shuffles
+// into 32-bit stores, so no CTA barrier is needed inside the loop. NVFP4 runs after
+// prep_mask_kernel and takes the mask from its metadata and the tensor amax from its
+// reduction; MXFP4 needs no tensor scale and computes the mask inline.
 //
 // Per unit the backbone is encoded at all 32 positions with the block's scale (its max
 // |x| is the unit's max |x|: the largest element of every group of 8 lies in its top pair,
@@ -185,96 +275,86 @@ __device__ float grid_amax(const uint4* __restrict__ X, size_t n16, AmaxState* s
 // at kept positions and +0 elsewhere, so r = x - deq needs no per-element selection.
 template <bool BF16, int FMT, bool RESIDUAL>
 __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
-  constexpr int RB = FMT == SHARQ_NVFP4 ? 16 : 32;  // residual block
+  constexpr bool NV = FMT == SHARQ_NVFP4;
+  constexpr int RB = NV ? 16 : 32;  // residual block
   __shared__ uint32_t s_top2[64];
+  __shared__ uint32_t s_nib[16];
+  __shared__ NvScaleTable s_nv;
+  __shared__ float s_amax;
   if (threadIdx.x < 64) s_top2[threadIdx.x] = top2_entry(threadIdx.x);
-
+  if (threadIdx.x < 16) s_nib[threadIdx.x] = nibble_entry(threadIdx.x);
+  // NVFP4: launched as a programmatic dependent of prep_mask_kernel; everything above runs
+  // while that kernel finishes, the wait below returns once its writes are visible
+  if (NV) asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (NV && threadIdx.x == 0) {
+    AmaxState* st = reinterpret_cast<AmaxState*>(p.tensor_scale + 2);
+    s_amax = __uint_as_float(*reinterpret_cast<volatile unsigned*>(&st->acc));
+    __threadfence();  // the read above completes before this CTA is counted
+    if (atomicAdd(&st->done, 1u) == gridDim.x - 1) {  // every CTA has read acc
+      st->acc = 0u;
+      st->done = 0u;
+    }
+  }
+  __syncthreads();
   TensorConsts tc{1.f, 1.f};
-  if (FMT == SHARQ_NVFP4) {
-    bool ok = true;
-    const float amax = grid_amax<BF16>(static_cast<const uint4*>(p.X),
-                                       size_t(p.M) * size_t(p.K) / 8,
-                                       reinterpret_cast<AmaxState*>(p.tensor_scale + 2),
-                                       p.status, p.timeout_ns, &ok);
-    if (!ok) return;
-    tc = tensor_consts(amax);
+  if constexpr (NV) {
+    tc = tensor_consts(s_amax);
+    nv_table_fill(&s_nv, tc.s_g, threadIdx.x);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
       p.tensor_scale[0] = tc.s_g;
-      p.tensor_scale[1] = amax;
+      p.tensor_scale[1] = s_amax;
     }
   } else if (blockIdx.x == 0 && threadIdx.x == 0) {
     p.tensor_scale[0] = 1.0f;
   }
-  __syncthreads();  // decision table ready
+  __syncthreads();  // decision and scale tables ready
 
-  const int K = p.K, M = p.M, Mp = p.Mp;
-  const int KS = K / 256;  // 256-K slices
-  const int n_items = (Mp / 4) * KS;
-  const int lane = threadIdx.x & 31;
-  const int u = lane & 7;    // 32-K unit inside the slice
-  const int rsub = lane >> 3;  // row inside the item
-  const int stride = gridDim.x * (blockDim.x >> 5);
-  const int stride_q = stride % KS, stride_r = (stride / KS) * 4;
-  const uint16_t* X = static_cast<const uint16_t*>(p.X);
-  const size_t scols_b = size_t(K) / 32 / 4;  // 512-byte chunks per 128 rows (backbone)
-  const size_t scols_r = size_t(K) / RB / 4;  // (residual)
+  const PairWalk wk(p);
+  const int K = wk.K, M = wk.M, u = wk.u;
+  const uint32_t scols_b = uint32_t(K) / 32 / 4;  // 512-byte chunks per 128 rows (backbone)
+  const uint32_t scols_r = uint32_t(K) / RB / 4;  // (residual)
 
-  int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  int q = item % KS;                // slice of the current item
-  int row = (item / KS) * 4 + rsub;  // row of this lane in the current item
-  uint4 cur[4];
-  auto load = [&](int it, int r, int qq, uint4* dst) {
-    if (it < n_items && r < M) {
-      const uint4* src =
-          reinterpret_cast<const uint4*>(X + size_t(r) * K + size_t(qq) * 256 + u * 32);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = __ldg(src + i);
-    }
+  // one block's scale; NVFP4 through the per-tensor table
+  auto scale_of = [&](float a) {
+    if constexpr (NV) return nv_block_scale(a, tc, &s_nv);
+    else return block_scale<FMT>(a, tc);
   };
-  load(item, row, q, cur);
+  auto decode_of = [&](uint32_t codes, const BlockScale& b, float* out) {
+    if constexpr (NV) decode8_nv(codes, b, tc.s_g, out);
+    else decode8<FMT>(codes, b, tc.s_g, out);
+  };
+  auto load_meta = [&](int it, int r, int q) -> uint32_t {
+    if (!NV || it >= wk.n_items || r >= M) return 0x4444u;
+    return __ldcg(reinterpret_cast<const unsigned short*>(wk.bm + wk.meta_off(q, r)));
+  };
+
+  int q = wk.q0, row = wk.row0;
+  uint4 cur[4];
+  wk.load(wk.first, row, q, cur);
+  uint32_t cmeta = load_meta(wk.first, row, q);
 
 #pragma unroll 1
-  for (; item < n_items; item += stride) {
-    int nq = q + stride_q, nrow = row + stride_r;
-    if (nq >= KS) {
-      nq -= KS;
-      nrow += 4;
-    }
+  for (int item = wk.first; item < wk.n_items; item += wk.stride) {
+    int nq = q, nrow = row;
+    wk.advance(nq, nrow);
     uint4 nxt[4];
-    load(item + stride, nrow, nq, nxt);
-    const int k0 = q * 256 + u * 32;
+    wk.load(item + wk.stride, nrow, nq, nxt);
+    const uint32_t nmeta = load_meta(item + wk.stride, nrow, nq);
+    const uint32_t k0 = uint32_t(q) * 256u + uint32_t(u) * 32u;
     const bool live = row < M;
-    uint32_t w[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      w[4 * i + 0] = cur[i].x; w[4 * i + 1] = cur[i].y;
-      w[4 * i + 2] = cur[i].z; w[4 * i + 3] = cur[i].w;
-    }
 
     uint32_t meta = 0x4444u, bsf = 0, rsf0 = 0, rsf1 = 0;
     if (live) {
-      // ---- mask: pair keys (max |x| << 16 | min |x|, as 15-bit magnitudes) and one
-      // table entry per group of 4 pairs; the comparison bits are the sign bits of
-      // key_j - key_i - 1, shifted in from (2,3) down to (0,1)
-      uint32_t L[4];
+      uint32_t w[16], L[4];
+      unpack16(cur, w);
+      if constexpr (NV) {
+        meta = cmeta;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t k[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t m = w[4 * g + j] & 0x7FFF7FFFu;
-          k[j] = max(m, __byte_perm(m, 0, 0x1032));
-        }
-        uint32_t idx = (k[3] - k[2] - 1u) >> 31;
-        idx = __funnelshift_l(k[3] - k[1] - 1u, idx, 1);
-        idx = __funnelshift_l(k[2] - k[1] - 1u, idx, 1);
-        idx = __funnelshift_l(k[3] - k[0] - 1u, idx, 1);
-        idx = __funnelshift_l(k[2] - k[0] - 1u, idx, 1);
-        idx = __funnelshift_l(k[1] - k[0] - 1u, idx, 1);
-        L[g] = s_top2[idx];
+        for (int g = 0; g < 4; ++g) L[g] = s_nib[(meta >> (4 * g)) & 0xFu];
+      } else {
+        uint32_t unused = 0;
+        meta = pair_mask(w, s_top2, L, &unused);
       }
-      meta = ((L[0] >> 24) & 0xFu) | ((L[1] >> 20) & 0xF0u) | ((L[2] >> 16) & 0xF00u) |
-             ((L[3] >> 12) & 0xF000u);
 
       float x[32];
 #pragma unroll
@@ -283,7 +363,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
         x[2 * i + 1] = hi16<BF16>(w[i]);
       }
       // ---- backbone: one block of 32 logical K
-      const BlockScale bb = block_scale<FMT>(amax_n<32>(x), tc);
+      const BlockScale bb = scale_of(amax_n<32>(x));
       bsf = bb.code;
       uint32_t c[4];
 #pragma unroll
@@ -292,7 +372,8 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
       // selector takes bytes i0, i1 of the first word and 4 + i0, 4 + i1 of the second)
       const uint32_t sel01 = __byte_perm(L[0], L[1], 0x0062u) + 0x4400u;
       const uint32_t sel23 = __byte_perm(L[2], L[3], 0x0062u) + 0x4400u;
-      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.bq) + size_t(row) * (K / 4) + k0 / 4) =
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.bq) +
+                                (uint32_t(row) * uint32_t(K / 4) + k0 / 4)) =
           make_uint2(__byte_perm(c[0], c[1], sel01), __byte_perm(c[2], c[3], sel23));
       if (RESIDUAL) {
         // ---- residual against the quantised backbone
@@ -300,7 +381,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           float d[8];
-          decode8<FMT>(__byte_perm(c[g], 0u, L[g]), bb, tc.s_g, d);
+          decode_of(__byte_perm(c[g], 0u, L[g]), bb, d);
 #pragma unroll
           for (int j = 0; j < 8; j += 2) {
             const float2 t = sub2_rn(make_float2(x[8 * g + j], x[8 * g + j + 1]),
@@ -312,18 +393,19 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
         uint32_t rc[4];
 #pragma unroll
         for (int hb = 0; hb < 32 / RB; ++hb) {
-          const BlockScale rb = block_scale<FMT>(amax_n<RB>(r + hb * RB), tc);
+          const BlockScale rb = scale_of(amax_n<RB>(r + hb * RB));
           if (hb == 0) rsf0 = rb.code; else rsf1 = rb.code;
 #pragma unroll
           for (int g = 0; g < RB / 8; ++g) rc[hb * (RB / 8) + g] = encode8(r + hb * RB + 8 * g, rb);
         }
-        *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.rq) + size_t(row) * (K / 2) + k0 / 2) =
+        *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.rq) +
+                                  (uint32_t(row) * uint32_t(K / 2) + k0 / 2)) =
             make_uint4(rc[0], rc[1], rc[2], rc[3]);
       }
     }
 
-    // ---- scales and metadata: gather neighbouring lanes' bytes into 32-bit stores
-    const size_t rq32 = size_t(row & 31) * 16 + size_t((row >> 5) & 3) * 4;
+    // ---- scales (and MXFP4 metadata): gather neighbouring lanes' bytes into 32-bit stores
+    const uint32_t rq32 = uint32_t(row & 31) * 16u + uint32_t((row >> 5) & 3) * 4u;
     {
       // backbone scale column q*8+u: lanes u..u+3 form one 4-byte word
       uint32_t word = bsf;
@@ -331,8 +413,8 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
       word |= __shfl_down_sync(0xFFFFFFFFu, bsf, 2) << 16;
       word |= __shfl_down_sync(0xFFFFFFFFu, bsf, 3) << 24;
       if ((u & 3) == 0) {
-        const size_t chunk = size_t(row >> 7) * scols_b + size_t(q) * 2 + size_t(u >> 2);
-        *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.bs) + chunk * 512 + rq32) = word;
+        const uint32_t chunk = uint32_t(row >> 7) * scols_b + uint32_t(q) * 2u + uint32_t(u >> 2);
+        *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.bs) + (chunk * 512u + rq32)) = word;
       }
     }
     if (RESIDUAL) {
@@ -341,8 +423,8 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
         const uint32_t two = rsf0 | (rsf1 << 8);
         const uint32_t word = two | (__shfl_down_sync(0xFFFFFFFFu, two, 1) << 16);
         if ((u & 1) == 0) {
-          const size_t chunk = size_t(row >> 7) * scols_r + size_t(q) * 4 + size_t(u >> 1);
-          *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.rs) + chunk * 512 + rq32) = word;
+          const uint32_t chunk = uint32_t(row >> 7) * scols_r + uint32_t(q) * 4u + uint32_t(u >> 1);
+          *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.rs) + (chunk * 512u + rq32)) = word;
         }
       } else {
         uint32_t word = rsf0;
@@ -350,25 +432,20 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
         word |= __shfl_down_sync(0xFFFFFFFFu, rsf0, 2) << 16;
         word |= __shfl_down_sync(0xFFFFFFFFu, rsf0, 3) << 24;
         if ((u & 3) == 0) {
-          const size_t chunk = size_t(row >> 7) * scols_r + size_t(q) * 2 + size_t(u >> 2);
-          *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.rs) + chunk * 512 + rq32) = word;
+          const uint32_t chunk = uint32_t(row >> 7) * scols_r + uint32_t(q) * 2u + uint32_t(u >> 2);
+          *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.rs) + (chunk * 512u + rq32)) = word;
         }
       }
     }
-    {
-      // metadata: 4 nibbles per lane, row's 16 bytes at slice q; lanes u, u+1 -> one word
-      const uint32_t m16 = meta & 0xFFFFu;
-      const uint32_t word = m16 | (__shfl_down_sync(0xFFFFFFFFu, m16, 1) << 16);
-      if ((u & 1) == 0)
-        *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.bm) + size_t(q) * Mp * 16 +
-                                     size_t(row) * 16 + u * 2) = word;
-    }
+    if constexpr (!NV) wk.store_meta(q, row, meta);
 #pragma unroll
     for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+    cmeta = nmeta;
     q = nq;
     row = nrow;
   }
 }
+
 
 // ------------------------------------------------------------------------------ element 2:4
 
@@ -529,18 +606,28 @@ static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cud
     if (per_sm == 0) {
       cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
       if (e != cudaSuccess) return e;
-      if (per_sm < 1) return cudaErrorInvalidConfiguration;
+      if (per_sm < 1) per_sm = 1;
     }
     const long items = long(p.Mp / 4) * (p.K / 256);
     long blocks = (items + 7) / 8;
     const long cap = long(num_sms) * per_sm;
     if (blocks > cap) blocks = cap;
     if (FMT == SHARQ_NVFP4) {
-      // the in-kernel tensor amax waits for every CTA: launch them all resident
-      PrepParams q = p;
-      void* args[] = {&q};
-      return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(unsigned(blocks)),
-                                         dim3(256), args, 0, st);
+      prep_mask_kernel<BF16><<<unsigned(blocks), 256, 0, st>>>(p);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      // programmatic dependent launch: the quantisation kernel's launch and prologue overlap
+      // the mask kernel
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(unsigned(blocks));
+      cfg.blockDim = dim3(256);
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      return cudaLaunchKernelEx(&cfg, kern, p);
     }
     kern<<<unsigned(blocks), 256, 0, st>>>(p);
   } else {

@@ -284,6 +284,9 @@ sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* a,
   sharq_status s = act_sizes(a->M, a->K, a->cfg, &sz);
   if (s != SHARQ_OK) return s;
   const bool res = a->cfg.residual == 1;
+  // the pair-mask kernel addresses X and its outputs with 32-bit offsets
+  if (a->cfg.mask == SHARQ_MASK_PAIR_4_8 && size_t(a->M) * size_t(a->K) >= (size_t(1) << 31))
+    return SHARQ_ERR_UNSUPPORTED;
   if (!a->bq || !a->bs || !a->bm || !a->tensor_scale || (res && (!a->rq || !a->rs)))
     return SHARQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(a->bq) || !aligned16(a->bs) || !aligned16(a->bm) ||

@@ -112,9 +112,9 @@ typedef struct {
   void* rs;            /* residual scales, tiled, M x K/residual_block */
   float* tensor_scale; /* 8 floats (32 bytes): [0] s_g = amax|X| / 2688 (NVFP4) or 1.0
                           (MXFP4); [1] amax|X| (NVFP4); both written by sharq_prepare.
-                          [2..7] library state of the in-kernel amax reduction: set them to
-                          zero once when the buffer is allocated and never write them
-                          afterwards (re-zero after a SHARQ_ERR_TIMEOUT). */
+                          [2..7] library state of the amax reduction: set them to zero once
+                          when the buffer is allocated and never write them afterwards
+                          (re-zero them if a call was interrupted by a device error). */
   int32_t M, K;
   sharq_config cfg;
 } sharq_act;
@@ -141,9 +141,10 @@ SHARQ_API sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, c
  * into one operator). X: device pointer to X[M x K] row-major in `dtype` (F16 or BF16).
  * Computes the tensor scale (NVFP4) in a first pass over X, then writes every buffer of
  * *act, including padding rows of the tiled scale and metadata layouts. With the pair
- * mask both passes run in one cooperative launch (a grid-wide wait, bounded in time:
- * on expiry the kernel records SHARQ_ERR_TIMEOUT for sharq_device_status); calls that
- * share one act->tensor_scale buffer must be ordered (one stream). */
+ * mask the first pass also computes the mask and metadata, and the second reads them back;
+ * the two kernels hand the tensor amax over through act->tensor_scale[2..3], so calls
+ * that share one act->tensor_scale buffer must be ordered (one stream). With the pair
+ * mask M * K must be below 2^31 (else SHARQ_ERR_UNSUPPORTED). */
 SHARQ_API sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* act, void* stream);
 
 /* Y[M x N] = alpha * (sparse-FP4-GEMM(backbone, W) + dense-FP4-GEMM(residual, W)) with

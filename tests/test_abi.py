@@ -109,6 +109,14 @@ def test_null_and_misaligned_pointers_rejected_before_any_launch(sq):
                            None) == 1  # bad out dtype
 
 
+def test_prepare_rejects_tensors_beyond_32_bit_offsets(sq):
+    p = ctypes.c_void_p
+    cfg = sq.Config().c()
+    act = sq.sharq_act(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), p(0x6000),
+                       65536, 32768, cfg)
+    assert sq.sharq_prepare(p(0x1000), sq.BF16, ctypes.byref(act), None) == 2
+
+
 def test_no_cpu_fallback_without_gpu(sq):
     """On a machine without a usable sm_100 GPU the compute calls return an error code
     (CUDA or ARCH) instead of computing anything on the host."""
