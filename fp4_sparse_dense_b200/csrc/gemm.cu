@@ -133,6 +133,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint64_t limit = p.timeout_ns;
+  // launched as a programmatic dependent: the set-up above overlapped the previous kernel;
+  // nothing it wrote (the operands) is read before this point
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -353,7 +357,18 @@ static cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, int num_sms,
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n * p.splits;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  kern<<<grid, kThreads, C::SMEM, st>>>(m.w, m.b, m.r, m.y, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, m.w, m.b, m.r, m.y, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -364,6 +379,7 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
                                                             int splits, int M, int N,
                                                             const float* act_ts, const float* w_ts,
                                                             void* Y) {
+  ptx::griddep_wait();  // the partials of the GEMM launched just before
   const size_t total = size_t(M) * N;
   const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
   if (i >= total) return;
@@ -436,10 +452,20 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int 
   if (e != cudaSuccess || p.splits <= 1) return e;
   const size_t total = size_t(p.M) * p.N;
   const unsigned blocks = unsigned((total / 8 + 255) / 256);
-  if (out_f32)
-    splitk_reduce_kernel<true><<<blocks, 256, 0, st>>>(p.ws, p.splits, p.M, p.N, p.act_ts, p.w_ts, p.Y);
-  else
-    splitk_reduce_kernel<false><<<blocks, 256, 0, st>>>(p.ws, p.splits, p.M, p.N, p.act_ts, p.w_ts, p.Y);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = out_f32 ? cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<true>, (const float*)p.ws, p.splits,
+                                   p.M, p.N, p.act_ts, p.w_ts, p.Y)
+              : cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<false>, (const float*)p.ws, p.splits,
+                                   p.M, p.N, p.act_ts, p.w_ts, p.Y);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -136,6 +136,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint64_t limit = p.timeout_ns;
+  // launched as a programmatic dependent: the set-up above overlapped the previous kernel;
+  // nothing it wrote (the operands) is read before this point
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   // the leader's copies of the barriers (the pair's loads and epilogues report there)
   const uint32_t lead_full0 = ptx::mapa(ptx::smem_u32(full_bar), 0);
   const uint32_t lead_tempty = ptx::mapa(ptx::smem_u32(tempty_bar), 0);
@@ -346,13 +350,15 @@ static cudaError_t launch_pair_t(const GemmPairMaps& m, const GemmParams& p, int
   cfg.blockDim = dim3(kPairThreads);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kern, m, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

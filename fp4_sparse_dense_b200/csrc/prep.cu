@@ -228,7 +228,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
   // the quantisation kernel may start its prologue now; it waits for this grid's completion
   // (griddepcontrol.wait) before it reads anything written here
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  ptx::griddep_launch_dependents();
   __shared__ uint32_t s_top2[64];
   if (threadIdx.x < 64) s_top2[threadIdx.x] = top2_entry(threadIdx.x);
   __syncthreads();
@@ -285,7 +285,8 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   if (threadIdx.x < 16) s_nib[threadIdx.x] = nibble_entry(threadIdx.x);
   // NVFP4: launched as a programmatic dependent of prep_mask_kernel; everything above runs
   // while that kernel finishes, the wait below returns once its writes are visible
-  if (NV) asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (NV) ptx::griddep_wait();
+  ptx::griddep_launch_dependents();  // the GEMM that follows may start its prologue
   if (NV && threadIdx.x == 0) {
     AmaxState* st = reinterpret_cast<AmaxState*>(p.tensor_scale + 2);
     s_amax = __uint_as_float(*reinterpret_cast<volatile unsigned*>(&st->acc));

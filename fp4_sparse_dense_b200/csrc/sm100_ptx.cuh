@@ -21,6 +21,16 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
+// Programmatic dependent launch (PTX griddepcontrol): a kernel launched with the
+// programmatic-stream-serialization attribute may start before the previous kernel in the
+// stream has finished; griddep_wait() returns once that kernel has completed and its memory
+// is visible (at once for a kernel launched without the attribute). griddep_launch_dependents()
+// lets the next such kernel start launching early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;
   asm volatile(

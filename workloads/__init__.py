@@ -39,11 +39,15 @@ def round_to_bf16(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     """
     x = np.ascontiguousarray(x, dtype=np.float32)
     assert np.all(np.isfinite(x))
-    b = x.view(np.uint32).astype(np.uint64)
-    lsb = (b >> 16) & 1
-    r = ((b + 0x7FFF + lsb) >> 16).astype(np.uint16)
-    vals = (r.astype(np.uint32) << 16).view(np.float32)
-    return vals, r
+    # uint32 arithmetic cannot overflow: finite patterns are <= 0xFF7FFFFF
+    b = x.view(np.uint32)
+    t = (b >> 16) & 1
+    t += 0x7FFF
+    t += b
+    t >>= 16
+    r = t.astype(np.uint16)
+    t <<= 16
+    return t.view(np.float32), r
 
 
 def round_to_f16(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
@@ -82,7 +86,9 @@ def _mk(x: np.ndarray, dtype: str) -> Tensor16:
 def gaussian_weight(rng: np.random.Generator, K: int, N: int, dtype: str = BF16,
                     sigma: float = 0.02) -> Tensor16:
     """W[K x N] ~ N(0, sigma^2): the layer's weight, input features along rows."""
-    return _mk(rng.normal(0.0, sigma, size=(K, N)).astype(np.float32), dtype)
+    w = rng.standard_normal((K, N), dtype=np.float32)
+    w *= np.float32(sigma)
+    return _mk(w, dtype)
 
 
 def tiny_activations(M: int = 16, K: int = 256, seed: int = 0, n_outliers: int = 4,
@@ -148,6 +154,8 @@ class Problem:
             return x, w
         rng = np.random.default_rng(self.seed)
         x = heavy_activations(rng, self.M, self.K, per_row=self.per_row, dtype=self.dtype)
+        if "w_seed" in self.extra:  # layer stack: each linear's weight has its own stream
+            rng = np.random.default_rng(100_000 + self.extra["w_seed"])
         w = gaussian_weight(rng, self.K, self.N, self.dtype)
         return x, w
 
