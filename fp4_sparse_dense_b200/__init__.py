@@ -20,11 +20,12 @@ from ._abi import (  # noqa: F401
     sharq_act, sharq_act_bytes, sharq_config, sharq_weight, sharq_weight_bytes, check,
     sharq_act_sizes, sharq_weight_sizes, sharq_status_string, sharq_device_status,
     sharq_prepare, sharq_quantize_weight, sharq_linear, sharq_linear_workspace_size,
-    sharq_linear_noalloc,
+    sharq_linear_noalloc, sharq_prepare_rmsnorm,
 )
 
 __all__ = [
-    "Config", "QuantWeight", "PreparedAct", "quantize_weight", "prepare", "linear",
+    "Config", "QuantWeight", "PreparedAct", "quantize_weight", "prepare", "prepare_rmsnorm",
+    "linear", "sharq_prepare_rmsnorm",
     "sharq_act_sizes", "sharq_weight_sizes", "sharq_prepare", "sharq_quantize_weight",
     "sharq_linear", "sharq_linear_workspace_size", "sharq_linear_noalloc", "sharq_device_status",
     "sharq_status_string", "SharqError", "linear_workspace",
@@ -147,6 +148,24 @@ def prepare(X, cfg: Config = Config(), out: PreparedAct | None = None, stream=No
     ca = out.c()
     check(sharq_prepare(_ptr(X), _dtype_code(X), ctypes.byref(ca), _stream(stream)))
     return out
+
+
+def prepare_rmsnorm(X, gamma, eps: float, cfg: Config = Config(), out: PreparedAct | None = None,
+                    rstd=None, stream=None):
+    """Prepare RMSNorm(X) with weight gamma [K] (same dtype as X): returns (act, rstd [M])."""
+    torch = _torch()
+    M, K = X.shape
+    X = X.contiguous()
+    gamma = gamma.contiguous()
+    if gamma.dtype != X.dtype or gamma.numel() != K:
+        raise ValueError("gamma must be [K] in the dtype of X")
+    out = out or empty_act(M, K, cfg, X.device)
+    if rstd is None:
+        rstd = torch.empty(M, dtype=torch.float32, device=X.device)
+    ca = out.c()
+    check(sharq_prepare_rmsnorm(_ptr(X), _ptr(gamma), float(eps), _dtype_code(X), _ptr(rstd),
+                                ctypes.byref(ca), _stream(stream)))
+    return out, rstd
 
 
 def linear_workspace(M: int, N: int, K: int, cfg: Config = Config(), device="cuda"):

@@ -58,6 +58,73 @@ __global__ void __launch_bounds__(512) amax_kernel(const uint4* __restrict__ X, 
   }
 }
 
+// ------------------------------------------------------------------------------ RMSNorm
+
+// Per-row rstd = 1 / sqrt(mean_k x^2 + eps), the RMSNorm that the preparation absorbs (the
+// SharQ page's fused operator takes in layer normalisation; RMSNorm is that of the
+// Llama/Qwen models it evaluates). One warp per row. The float32 order is fixed so that the
+// result is reproducible: chunk c of 8 elements belongs to lane c mod 32, each lane adds
+// its chunks' squares in increasing k, then a butterfly over lanes (xor 16, 8, 4, 2, 1).
+// Squares of 16-bit inputs are exact; every addition and the division, square root and
+// reciprocal round to nearest once.
+template <bool BF16>
+__global__ void __launch_bounds__(256) rms_kernel(PrepParams p) {
+  ptx::griddep_wait();  // X may come from the kernel launched just before
+  ptx::griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const uint32_t chunks = uint32_t(p.K) / 8;
+  for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < p.M; row += warps) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.X) +
+                                                      uint32_t(row) * uint32_t(p.K));
+    float acc = 0.f;
+#pragma unroll 4
+    for (uint32_t c = lane; c < chunks; c += 32) {
+      const uint4 v = __ldg(src + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = in_to_float<BF16>(w[i] & 0xFFFFu), hi = in_to_float<BF16>(w[i] >> 16);
+        acc = __fadd_rn(acc, __fmul_rn(lo, lo));
+        acc = __fadd_rn(acc, __fmul_rn(hi, hi));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xFFFFFFFFu, acc, off));
+    if (lane == 0) {
+      const float ms = __fdiv_rn(acc, float(p.K));
+      p.rstd[row] = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, p.eps)));
+    }
+  }
+}
+
+// y = round16((x * rstd) * gamma) for the 32 inputs of one unit (16 words of two 16-bit
+// values, k0 the unit's first column): the normalised input the preparation then sees.
+template <bool BF16>
+__device__ __forceinline__ void rms_apply(uint32_t* w, const PrepParams& p, int row,
+                                          uint32_t k0) {
+  const float r = __ldg(p.rstd + row);
+  const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.gamma) + k0);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 gv = __ldg(g4 + c);
+    const uint32_t g[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t& x = w[4 * c + i];
+      const float lo = __fmul_rn(__fmul_rn(in_to_float<BF16>(x & 0xFFFFu), r),
+                                 in_to_float<BF16>(g[i] & 0xFFFFu));
+      const float hi = __fmul_rn(__fmul_rn(in_to_float<BF16>(x >> 16), r),
+                                 in_to_float<BF16>(g[i] >> 16));
+      if (BF16) {
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(x) : "f"(hi), "f"(lo));
+      } else {
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(x) : "f"(hi), "f"(lo));
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------ pair 4:8
 
 // Entry of the top-2-of-4 decision table. Bit b of `idx` is one comparison "candidate i
@@ -224,7 +291,7 @@ __device__ __forceinline__ void unpack16(const uint4* c, uint32_t* w) {
 // First NVFP4 preparation kernel (pair mask): streams X from HBM, computes the mask, writes
 // the metadata (padding rows included) and folds max |x| into the tensor amax. Its integer
 // work hides under the HBM reads.
-template <bool BF16>
+template <bool BF16, bool NORM>
 __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
   // the quantisation kernel may start its prologue now; it waits for this grid's completion
   // (griddepcontrol.wait) before it reads anything written here
@@ -232,6 +299,7 @@ __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
   __shared__ uint32_t s_top2[64];
   if (threadIdx.x < 64) s_top2[threadIdx.x] = top2_entry(threadIdx.x);
   __syncthreads();
+  ptx::griddep_wait();  // X (and rstd) come from the kernels launched before
   const PairWalk wk(p);
   uint32_t mx = 0;
   int q = wk.q0, row = wk.row0;
@@ -247,6 +315,7 @@ __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
     if (row < wk.M) {
       uint32_t w[16], L[4];
       unpack16(cur, w);
+      if (NORM) rms_apply<BF16>(w, p, row, uint32_t(q) * 256u + uint32_t(wk.u) * 32u);
       meta = pair_mask(w, s_top2, L, &mx);
     }
     wk.store_meta(q, row, meta);
@@ -273,7 +342,7 @@ __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
 // which is kept); byte permutes then keep the kept pairs' code bytes, either compressed
 // (the backbone operand) or in place with zeros elsewhere, which dequantise to the backbone
 // at kept positions and +0 elsewhere, so r = x - deq needs no per-element selection.
-template <bool BF16, int FMT, bool RESIDUAL>
+template <bool BF16, int FMT, bool RESIDUAL, bool NORM>
 __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   constexpr bool NV = FMT == SHARQ_NVFP4;
   constexpr int RB = NV ? 16 : 32;  // residual block
@@ -285,7 +354,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   if (threadIdx.x < 16) s_nib[threadIdx.x] = nibble_entry(threadIdx.x);
   // NVFP4: launched as a programmatic dependent of prep_mask_kernel; everything above runs
   // while that kernel finishes, the wait below returns once its writes are visible
-  if (NV) ptx::griddep_wait();
+  ptx::griddep_wait();
   ptx::griddep_launch_dependents();  // the GEMM that follows may start its prologue
   if (NV && threadIdx.x == 0) {
     AmaxState* st = reinterpret_cast<AmaxState*>(p.tensor_scale + 2);
@@ -348,6 +417,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
     if (live) {
       uint32_t w[16], L[4];
       unpack16(cur, w);
+      if (NORM) rms_apply<BF16>(w, p, row, k0);
       if constexpr (NV) {
         meta = cmeta;
 #pragma unroll
@@ -599,10 +669,27 @@ __global__ void __launch_bounds__(256) prep_elem_kernel(PrepParams p) {
 
 // ------------------------------------------------------------------------------ launch
 
-template <bool BF16, int FMT, bool RES>
+// launch with the programmatic-stream-serialization attribute: the kernel may start while
+// the previous one in the stream finishes and waits (griddepcontrol.wait) for its results
+template <typename... Args>
+static cudaError_t launch_pdl(void (*kern)(Args...), unsigned blocks, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+template <bool BF16, int FMT, bool RES, bool NORM>
 static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
   if (mask == SHARQ_MASK_PAIR_4_8) {
-    auto kern = prep_pair_kernel<BF16, FMT, RES>;
+    auto kern = prep_pair_kernel<BF16, FMT, RES, NORM>;
     static int per_sm = 0;  // resident CTAs per SM (one value per instantiation)
     if (per_sm == 0) {
       cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
@@ -613,42 +700,45 @@ static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cud
     long blocks = (items + 7) / 8;
     const long cap = long(num_sms) * per_sm;
     if (blocks > cap) blocks = cap;
-    if (FMT == SHARQ_NVFP4) {
-      prep_mask_kernel<BF16><<<unsigned(blocks), 256, 0, st>>>(p);
-      cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaSuccess;
+    if (NORM) {  // per-row rstd first: one warp per row
+      long rb = (long(p.M) + 7) / 8;
+      if (rb > long(num_sms) * 8) rb = long(num_sms) * 8;
+      e = launch_pdl(rms_kernel<BF16>, unsigned(rb), st, p);
       if (e != cudaSuccess) return e;
-      // programmatic dependent launch: the quantisation kernel's launch and prologue overlap
-      // the mask kernel
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(unsigned(blocks));
-      cfg.blockDim = dim3(256);
-      cfg.stream = st;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      return cudaLaunchKernelEx(&cfg, kern, p);
     }
-    kern<<<unsigned(blocks), 256, 0, st>>>(p);
+    if (FMT == SHARQ_NVFP4) {
+      e = launch_pdl(prep_mask_kernel<BF16, NORM>, unsigned(blocks), st, p);
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_pdl(kern, unsigned(blocks), st, p);
+    if (e != cudaSuccess) return e;
   } else {
+    if (NORM) return cudaErrorNotSupported;
     dim3 grid(p.K / 256, (p.M + 127) / 128);
     prep_elem_kernel<BF16, FMT, RES><<<grid, 256, 0, st>>>(p);
   }
   return cudaGetLastError();
 }
 
+template <bool BF16, int FMT, bool RES>
+static cudaError_t launch_prep_n(const PrepParams& p, int mask, bool norm, int n, cudaStream_t st) {
+  return norm ? launch_prep_t<BF16, FMT, RES, true>(p, mask, n, st)
+              : launch_prep_t<BF16, FMT, RES, false>(p, mask, n, st);
+}
+
 template <bool BF16, int FMT>
-static cudaError_t launch_prep_r(const PrepParams& p, int mask, bool res, int n, cudaStream_t st) {
-  return res ? launch_prep_t<BF16, FMT, true>(p, mask, n, st)
-             : launch_prep_t<BF16, FMT, false>(p, mask, n, st);
+static cudaError_t launch_prep_r(const PrepParams& p, int mask, bool res, bool norm, int n,
+                                 cudaStream_t st) {
+  return res ? launch_prep_n<BF16, FMT, true>(p, mask, norm, n, st)
+             : launch_prep_n<BF16, FMT, false>(p, mask, norm, n, st);
 }
 
 template <bool BF16>
-static cudaError_t launch_prep_f(const PrepParams& p, int fmt, int mask, bool res, int n,
-                                 cudaStream_t st) {
-  return fmt == SHARQ_NVFP4 ? launch_prep_r<BF16, SHARQ_NVFP4>(p, mask, res, n, st)
-                            : launch_prep_r<BF16, SHARQ_MXFP4>(p, mask, res, n, st);
+static cudaError_t launch_prep_f(const PrepParams& p, int fmt, int mask, bool res, bool norm,
+                                 int n, cudaStream_t st) {
+  return fmt == SHARQ_NVFP4 ? launch_prep_r<BF16, SHARQ_NVFP4>(p, mask, res, norm, n, st)
+                            : launch_prep_r<BF16, SHARQ_MXFP4>(p, mask, res, norm, n, st);
 }
 
 cudaError_t launch_amax(const void* X, bool bf16, size_t n_elems, unsigned int* amax_bits,
@@ -667,8 +757,9 @@ cudaError_t launch_amax(const void* X, bool bf16, size_t n_elems, unsigned int* 
 
 cudaError_t launch_prep(const PrepParams& p, bool bf16, int fmt, int mask, bool residual,
                         int num_sms, cudaStream_t st) {
-  return bf16 ? launch_prep_f<true>(p, fmt, mask, residual, num_sms, st)
-              : launch_prep_f<false>(p, fmt, mask, residual, num_sms, st);
+  const bool norm = p.gamma != nullptr;
+  return bf16 ? launch_prep_f<true>(p, fmt, mask, residual, norm, num_sms, st)
+              : launch_prep_f<false>(p, fmt, mask, residual, norm, num_sms, st);
 }
 
 }  // namespace sharq

@@ -219,6 +219,67 @@ sharq_status weight_sizes(int32_t K, int32_t N, sharq_config c, sharq_weight_byt
 
 using namespace sharq;
 
+namespace sharq {
+namespace {
+// Both preparation entry points: gamma == nullptr prepares X as given; otherwise the
+// RMSNorm of X with (gamma, eps), writing the per-row rstd.
+sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, const void* gamma,
+                          float eps, float* rstd, void* stream) {
+  if (!X || !a) return SHARQ_ERR_INVALID_ARG;
+  if (dtype != SHARQ_F16 && dtype != SHARQ_BF16) return SHARQ_ERR_INVALID_ARG;
+  sharq_act_bytes sz;
+  sharq_status s = act_sizes(a->M, a->K, a->cfg, &sz);
+  if (s != SHARQ_OK) return s;
+  const bool res = a->cfg.residual == 1;
+  const bool norm = gamma != nullptr;
+  if (norm && a->cfg.mask != SHARQ_MASK_PAIR_4_8) return SHARQ_ERR_UNSUPPORTED;
+  // the pair-mask kernels address X and their outputs with 32-bit offsets
+  if (a->cfg.mask == SHARQ_MASK_PAIR_4_8 && size_t(a->M) * size_t(a->K) >= (size_t(1) << 31))
+    return SHARQ_ERR_UNSUPPORTED;
+  if (!a->bq || !a->bs || !a->bm || !a->tensor_scale || (res && (!a->rq || !a->rs)) ||
+      (norm && !rstd))
+    return SHARQ_ERR_INVALID_ARG;
+  if (norm && !(eps >= 0.f && eps < 1e30f)) return SHARQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(a->bq) || !aligned16(a->bs) || !aligned16(a->bm) ||
+      !aligned16(a->tensor_scale) || (res && (!aligned16(a->rq) || !aligned16(a->rs))) ||
+      (norm && (!aligned16(gamma) || !aligned16(rstd))))
+    return SHARQ_ERR_MISALIGNED;
+  DeviceInfo d;
+  if ((s = device_info(&d)) != SHARQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == SHARQ_BF16;
+  // the pair-mask kernels reduce the NVFP4 tensor amax themselves (state in
+  // tensor_scale[2..3]); the element-mask kernel takes it from a separate pass into
+  // tensor_scale[1]
+  if (a->cfg.fmt == SHARQ_NVFP4 && a->cfg.mask == SHARQ_MASK_ELEM_2_4) {
+    if (cudaMemsetAsync(a->tensor_scale + 1, 0, sizeof(float), st) != cudaSuccess)
+      return SHARQ_ERR_CUDA;
+    s = from_cuda(launch_amax(X, bf16, size_t(a->M) * size_t(a->K),
+                              reinterpret_cast<unsigned int*>(a->tensor_scale + 1), d.num_sms, st));
+    if (s != SHARQ_OK) return s;
+  }
+  PrepParams p;
+  p.X = X;
+  p.bq = a->bq;
+  p.bs = a->bs;
+  p.bm = a->bm;
+  p.rq = a->rq;
+  p.rs = a->rs;
+  p.tensor_scale = a->tensor_scale;
+  p.amax = a->tensor_scale + 1;
+  p.M = a->M;
+  p.K = a->K;
+  p.Mp = int(round_up(size_t(a->M), 128));
+  p.status = d.status;
+  p.timeout_ns = kWaitLimitNs;
+  p.gamma = gamma;
+  p.rstd = rstd;
+  p.eps = eps;
+  return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
+}
+}  // namespace
+}  // namespace sharq
+
 extern "C" {
 
 const char* sharq_status_string(sharq_status s) {
@@ -278,48 +339,13 @@ sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, const sharq
 }
 
 sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* a, void* stream) {
-  if (!X || !a) return SHARQ_ERR_INVALID_ARG;
-  if (dtype != SHARQ_F16 && dtype != SHARQ_BF16) return SHARQ_ERR_INVALID_ARG;
-  sharq_act_bytes sz;
-  sharq_status s = act_sizes(a->M, a->K, a->cfg, &sz);
-  if (s != SHARQ_OK) return s;
-  const bool res = a->cfg.residual == 1;
-  // the pair-mask kernel addresses X and its outputs with 32-bit offsets
-  if (a->cfg.mask == SHARQ_MASK_PAIR_4_8 && size_t(a->M) * size_t(a->K) >= (size_t(1) << 31))
-    return SHARQ_ERR_UNSUPPORTED;
-  if (!a->bq || !a->bs || !a->bm || !a->tensor_scale || (res && (!a->rq || !a->rs)))
-    return SHARQ_ERR_INVALID_ARG;
-  if (!aligned16(X) || !aligned16(a->bq) || !aligned16(a->bs) || !aligned16(a->bm) ||
-      !aligned16(a->tensor_scale) || (res && (!aligned16(a->rq) || !aligned16(a->rs))))
-    return SHARQ_ERR_MISALIGNED;
-  DeviceInfo d;
-  if ((s = device_info(&d)) != SHARQ_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool bf16 = dtype == SHARQ_BF16;
-  // the pair-mask kernel reduces the NVFP4 tensor amax itself (state in tensor_scale[2..5]);
-  // the element-mask kernel takes it from a separate pass into tensor_scale[1]
-  if (a->cfg.fmt == SHARQ_NVFP4 && a->cfg.mask == SHARQ_MASK_ELEM_2_4) {
-    if (cudaMemsetAsync(a->tensor_scale + 1, 0, sizeof(float), st) != cudaSuccess)
-      return SHARQ_ERR_CUDA;
-    s = from_cuda(launch_amax(X, bf16, size_t(a->M) * size_t(a->K),
-                              reinterpret_cast<unsigned int*>(a->tensor_scale + 1), d.num_sms, st));
-    if (s != SHARQ_OK) return s;
-  }
-  PrepParams p;
-  p.X = X;
-  p.bq = a->bq;
-  p.bs = a->bs;
-  p.bm = a->bm;
-  p.rq = a->rq;
-  p.rs = a->rs;
-  p.tensor_scale = a->tensor_scale;
-  p.amax = a->tensor_scale + 1;
-  p.M = a->M;
-  p.K = a->K;
-  p.Mp = int(round_up(size_t(a->M), 128));
-  p.status = d.status;
-  p.timeout_ns = kWaitLimitNs;
-  return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
+  return sharq::prepare_impl(X, dtype, a, nullptr, 0.f, nullptr, stream);
+}
+
+sharq_status sharq_prepare_rmsnorm(const void* X, const void* gamma, float eps, sharq_dtype dtype,
+                                   float* rstd, const sharq_act* a, void* stream) {
+  if (!gamma) return SHARQ_ERR_INVALID_ARG;
+  return sharq::prepare_impl(X, dtype, a, gamma, eps, rstd, stream);
 }
 
 sharq_status sharq_linear_workspace_size(int32_t M, int32_t N, int32_t K, sharq_config cfg,

@@ -21,6 +21,10 @@ struct PrepParams {
   int M, K, Mp;
   unsigned* status;     // device status word (bounded-wait timeouts)
   unsigned long long timeout_ns;
+  // RMSNorm absorbed into the preparation (null gamma: X is prepared as given)
+  const void* gamma;    // [K] 16-bit, same dtype as X
+  float* rstd;          // [M] per-row 1 / sqrt(mean x^2 + eps), written by rms_kernel
+  float eps;
 };
 
 struct WeightQuantParams {

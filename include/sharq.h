@@ -147,6 +147,20 @@ SHARQ_API sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, c
  * mask M * K must be below 2^31 (else SHARQ_ERR_UNSUPPORTED). */
 SHARQ_API sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* act, void* stream);
 
+/* Preparation with the layer's RMSNorm absorbed (SharQ page, abstract: the fused
+ * preparation operator takes in layer normalisation; RMSNorm is that of the Llama/Qwen
+ * models the page evaluates). The prepared input is y = round16((x * rstd) * gamma) per
+ * element, rstd = 1 / sqrt(mean_k x^2 + eps) per row, and *act is filled exactly as
+ * sharq_prepare(y) would fill it. Float32 throughout, one rounding per operation; the sum
+ * of squares in a fixed order (chunk c of 8 elements to accumulator c mod 32, in increasing
+ * k; then accumulators combined by xor 16, 8, 4, 2, 1), so results are reproducible.
+ * X: device [M x K] row-major in `dtype` (F16 or BF16, 16-byte aligned); gamma: device [K]
+ * in the same dtype; eps >= 0; rstd: device float[M], written. Pair mask only (element mask:
+ * SHARQ_ERR_UNSUPPORTED); M * K < 2^31. Nothing is written to X. */
+SHARQ_API sharq_status sharq_prepare_rmsnorm(const void* X, const void* gamma, float eps,
+                                             sharq_dtype dtype, float* rstd,
+                                             const sharq_act* act, void* stream);
+
 /* Y[M x N] = alpha * (sparse-FP4-GEMM(backbone, W) + dense-FP4-GEMM(residual, W)) with
  * alpha = s_g * s_gw, accumulated in FP32 tensor memory and written once (SharQ page, "Core
  * claim": a sparse FP4 GEMM for the backbone and a dense FP4 GEMM for the compensation,

@@ -117,6 +117,20 @@ def test_prepare_rejects_tensors_beyond_32_bit_offsets(sq):
     assert sq.sharq_prepare(p(0x1000), sq.BF16, ctypes.byref(act), None) == 2
 
 
+def test_prepare_rmsnorm_argument_checks(sq):
+    p = ctypes.c_void_p
+    act = sq.sharq_act(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), p(0x6000),
+                       16, 256, sq.Config().c())
+    f = sq.sharq_prepare_rmsnorm
+    assert f(p(0x1000), None, 1e-6, sq.BF16, p(0x7000), ctypes.byref(act), None) == 1  # gamma
+    assert f(p(0x1000), p(0x8000), 1e-6, sq.BF16, None, ctypes.byref(act), None) == 1  # rstd
+    assert f(p(0x1000), p(0x8000), -1.0, sq.BF16, p(0x7000), ctypes.byref(act), None) == 1
+    assert f(p(0x1000), p(0x8004), 1e-6, sq.BF16, p(0x7000), ctypes.byref(act), None) == 3
+    elem = sq.sharq_act(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), p(0x6000),
+                        16, 256, sq.Config.from_names("nvfp4", "elem24").c())
+    assert f(p(0x1000), p(0x8000), 1e-6, sq.BF16, p(0x7000), ctypes.byref(elem), None) == 2
+
+
 def test_no_cpu_fallback_without_gpu(sq):
     """On a machine without a usable sm_100 GPU the compute calls return an error code
     (CUDA or ARCH) instead of computing anything on the host."""
