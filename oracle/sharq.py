@@ -55,6 +55,15 @@ NVFP4 = "nvfp4"
 MXFP4 = "mxfp4"
 PAIR48 = "pair48"
 ELEM24 = "elem24"
+# ablation modes (the page's referee asks for them; see prepare): the pair-wise 4:8 mask
+# supplied by the caller (e.g. a static, per-tensor channel set) and no mask (plain FP4)
+PAIR48_GIVEN = "pair48_given"
+NONE = "none"
+
+
+def is_pair(mask: str) -> bool:
+    """Masks whose backbone is stored compressed and runs through the sparse MMA."""
+    return mask in (PAIR48, PAIR48_GIVEN)
 
 F32 = np.float32
 GLOBAL_DIV = F32(6.0 * 448.0)  # E2M1 max * E4M3 max
@@ -69,7 +78,7 @@ def residual_block(fmt: str) -> int:
 
 def backbone_block(fmt: str, mask: str) -> int:
     """Logical K positions covered by one backbone scale."""
-    if mask == PAIR48:
+    if is_pair(mask):
         return 32
     return residual_block(fmt)
 
@@ -77,7 +86,7 @@ def backbone_block(fmt: str, mask: str) -> int:
 def weight_block(fmt: str, mask: str) -> int:
     if fmt == MXFP4:
         return 32
-    return 32 if mask == PAIR48 else 16
+    return 32 if is_pair(mask) else 16
 
 
 def dense_view_block(fmt: str) -> int:
@@ -205,18 +214,40 @@ def keep_elems24(x: np.ndarray) -> np.ndarray:
     return _top2_of_4(a, np.zeros_like(a))
 
 
-def keep_mask(x: np.ndarray, mask: str) -> np.ndarray:
-    """Boolean [M, K]: True where the backbone keeps the element."""
+def static_keep_pairs48(x_stat: np.ndarray, M: int) -> np.ndarray:
+    """Static pair-wise 4:8 mask (ablation: the channel set fixed per tensor instead of
+    chosen per row): the pairs are ranked as in keep_pairs48, but on the per-column max |x|
+    of the statistics tensor x_stat, and the same kept pairs serve all M rows.
+    Boolean [M, K/8, 4]."""
+    col = np.max(np.abs(np.asarray(x_stat, F32)), axis=0, keepdims=True)  # [1, K]
+    return np.broadcast_to(keep_pairs48(col), (M,) + keep_pairs48(col).shape[1:]).copy()
+
+
+def keep_mask(x: np.ndarray, mask: str, given=None) -> np.ndarray:
+    """Boolean [M, K]: True where the backbone keeps the element. `given` is the kept pairs
+    ([M, K/8, 4]) of the pair48_given mode."""
     M, K = x.shape
     if mask == PAIR48:
         return np.repeat(keep_pairs48(x), 2, axis=-1).reshape(M, K)
+    if mask == PAIR48_GIVEN:
+        assert given is not None and np.all(np.asarray(given).sum(axis=-1) == 2)
+        return np.repeat(np.asarray(given, bool), 2, axis=-1).reshape(M, K)
+    if mask == NONE:
+        return np.ones((M, K), bool)
     return keep_elems24(x).reshape(M, K)
 
 
-def canonical_metadata(x: np.ndarray, mask: str) -> np.ndarray:
+def canonical_metadata(x: np.ndarray, mask: str, given=None) -> np.ndarray:
     """One nibble per group: i0 | i1 << 2 with i0 < i1 the kept pair indices (pair48)
-    or kept element indices (elem24). Shape [M, groups]."""
-    kept = keep_pairs48(x) if mask == PAIR48 else keep_elems24(x)
+    or kept element indices (elem24). Shape [M, groups]; empty for the "none" mode."""
+    if mask == NONE:
+        return np.zeros((x.shape[0], 0), np.uint8)
+    if mask == PAIR48:
+        kept = keep_pairs48(x)
+    elif mask == PAIR48_GIVEN:
+        kept = np.asarray(given, bool)
+    else:
+        kept = keep_elems24(x)
     pos = np.arange(4)
     i0 = np.where(kept, pos, 9).min(axis=-1)
     i1 = np.where(kept, pos, -1).max(axis=-1)
@@ -246,13 +277,18 @@ class Prepared:
 
 
 def prepare(x: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48, residual: bool = True,
-            residual_ref: str = "quantized", amax: np.float32 | None = None) -> Prepared:
+            residual_ref: str = "quantized", amax: np.float32 | None = None,
+            given=None) -> Prepared:
     """Online sparse-dense decomposition of one activation tensor X[M x K].
 
     residual_ref="quantized" is the method (r = x - deq(Q(backbone))); "unquantized"
-    is the ablation the page's referee asks for (r = x - backbone). `amax` overrides the
-    tensor's max |x|, so that a sample of rows can be prepared exactly as inside the
-    whole tensor (rows are independent once the tensor constants are fixed).
+    is the ablation the page's referee asks for (r = x - backbone: zero at kept
+    positions). The other referee ablations are masks: "pair48_given" takes the kept
+    pairs from `given` (a static mask, e.g. static_keep_pairs48), and "none" keeps every
+    element (plain FP4 of x in the residual's block size; with residual on, r = x -
+    deq(Q(x)) is a second, dense FP4 term). `amax` overrides the tensor's max |x|, so
+    that a sample of rows can be prepared exactly as inside the whole tensor (rows are
+    independent once the tensor constants are fixed).
     """
     x = np.ascontiguousarray(x, dtype=F32)
     M, K = x.shape
@@ -262,10 +298,10 @@ def prepare(x: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48, residual: bool 
     else:
         sc = (F32(1.0), F32(1.0))
     s_g = sc[0]
-    keep = keep_mask(x, mask)
-    meta = canonical_metadata(x, mask)
+    keep = keep_mask(x, mask, given)
+    meta = canonical_metadata(x, mask, given)
     Bb = backbone_block(fmt, mask)
-    if mask == PAIR48:
+    if is_pair(mask):
         comp = x[keep].reshape(M, K // 2)  # kept values in K order (row-major boolean gather)
         codes, bs, deq_c = quant_blocks(fmt, comp.reshape(M, -1, 16), sc)
         bq = codes.reshape(M, K // 2)
@@ -341,7 +377,7 @@ def backbone_values(p: Prepared) -> np.ndarray:
     Bb = backbone_block(p.fmt, p.mask)
     sv = scale_value(p.fmt, p.bs)  # [M, K/Bb]
     out = np.zeros((M, K))
-    if p.mask == PAIR48:
+    if is_pair(p.mask):
         vals = F.e2m1_decode(p.bq).reshape(M, K // Bb, 16) * sv[..., None]
         out[p.keep] = vals.reshape(-1)
     else:
@@ -399,9 +435,9 @@ def act_buffers(p: Prepared) -> dict:
     out = {"tensor_scale": np.array([p.s_g], F32)}
     out["bq"] = L.pack_nibbles(p.bq).reshape(-1)
     out["bs"] = L.to_scale_layout(p.bs)
-    if p.mask == PAIR48:
+    if is_pair(p.mask):
         out["bm"] = L.to_meta48_layout(p.meta)
-    else:
+    elif p.mask == ELEM24:
         out["bm"] = L.to_meta24_layout(p.meta)
     if p.residual:
         out["rq"] = L.pack_nibbles(p.rq).reshape(-1)
@@ -415,6 +451,6 @@ def weight_buffers(qw: QWeight) -> dict:
     out = {"tensor_scale": np.array([qw.s_gw], F32)}
     out["codes"] = L.pack_nibbles(qw.wq).reshape(-1)
     out["scales_dense"] = L.to_scale_layout(weight_scale_view(qw, dense_view_block(qw.fmt)))
-    if qw.mask == PAIR48:
+    if is_pair(qw.mask):
         out["scales_sparse"] = L.to_scale_layout(weight_scale_view(qw, SPARSE_VIEW_BLOCK))
     return out

@@ -1,0 +1,89 @@
+"""Pins of the oracle's ablation modes (the page's referee asks for a residual against the
+unquantised sparse values, a static instead of an input-adaptive mask, and direct FP4
+without the decomposition): closed forms, equivalences between independent code paths,
+and the direction of the reconstruction errors on outlier-heavy inputs."""
+import numpy as np
+import pytest
+
+from oracle import sharq as S
+from workloads import heavy_activations
+
+F32 = np.float32
+
+
+def _x(M=64, K=512, seed=0, per_row=True):
+    return heavy_activations(np.random.default_rng(seed), M, K, per_row=per_row).values
+
+
+def _recon(p):
+    """float64 reconstruction deq(backbone) + deq(residual) in the tensor's units."""
+    out = S.backbone_values(p) * float(p.s_g if p.fmt == S.NVFP4 else 1.0)
+    if p.residual:
+        out = out + p.r_deq.astype(np.float64)
+    return out
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_given_mask_equal_to_adaptive_reproduces_the_method(fmt):
+    x = _x()
+    a = S.act_buffers(S.prepare(x, fmt, S.PAIR48))
+    b = S.act_buffers(S.prepare(x, fmt, S.PAIR48_GIVEN, given=S.keep_pairs48(x)))
+    assert a.keys() == b.keys()
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_static_mask_equals_adaptive_when_rows_repeat():
+    row = _x(1, 512, seed=3)
+    x = np.repeat(row, 8, axis=0)
+    assert np.array_equal(S.static_keep_pairs48(x, 8), S.keep_pairs48(x))
+
+
+def test_static_mask_keeps_two_pairs_everywhere_and_the_same_in_every_row():
+    x = _x(32, 1024, seed=4)
+    g = S.static_keep_pairs48(x, 32)
+    assert np.all(g.sum(axis=-1) == 2)
+    assert np.all(g == g[:1])
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_unquantized_reference_residual_is_the_masked_out_part(fmt):
+    """r = x - backbone: exactly 0 where the mask keeps, exactly x elsewhere."""
+    x = _x(seed=5)
+    p = S.prepare(x, fmt, S.PAIR48, residual_ref="unquantized")
+    assert np.all(p.r[p.keep] == 0)
+    assert np.array_equal(p.r[~p.keep], x[~p.keep])
+
+
+def test_no_mask_equals_element_mask_when_groups_hold_two_nonzeros():
+    """With at most two non-zeros in every 4-group, the 2:4 backbone is all of x, so its
+    FP4 values equal plain FP4 of x (independent paths: the 2:4 selection vs keep-all)."""
+    rng = np.random.default_rng(6)
+    x = _x(32, 512, seed=6)
+    z = np.zeros_like(x).reshape(32, -1, 4)
+    for g in range(z.shape[1]):
+        cols = rng.choice(4, 2, replace=False)
+        z[:, g, cols] = 1
+    x = (x * z.reshape(x.shape)).astype(F32)
+    for fmt in ("nvfp4", "mxfp4"):
+        a = S.prepare(x, fmt, S.NONE, residual=False)
+        b = S.prepare(x, fmt, S.ELEM24, residual=False)
+        assert np.array_equal(S.backbone_values(a), S.backbone_values(b))
+        assert np.array_equal(a.bs, b.bs)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_ablation_error_ordering_on_outlier_heavy_inputs(fmt):
+    """Reconstruction error (Frobenius): the method <= each ablation on per-row outliers;
+    plain FP4 with a dense FP4 residual (two dense terms) <= plain FP4 alone."""
+    x = _x(256, 1024, seed=7, per_row=True)
+    err = lambda p: np.linalg.norm(x - _recon(p))
+    method = err(S.prepare(x, fmt, S.PAIR48))
+    unq = err(S.prepare(x, fmt, S.PAIR48, residual_ref="unquantized"))
+    static = err(S.prepare(x, fmt, S.PAIR48_GIVEN, given=S.static_keep_pairs48(x, 256)))
+    plain = err(S.prepare(x, fmt, S.NONE, residual=False))
+    plain2 = err(S.prepare(x, fmt, S.NONE, residual=True))
+    assert method <= unq
+    assert method <= static
+    assert method <= plain
+    assert plain2 <= plain
