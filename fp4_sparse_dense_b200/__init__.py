@@ -16,7 +16,8 @@ import os
 from dataclasses import dataclass
 
 from ._abi import (  # noqa: F401
-    ELEM_2_4, F16, F32, BF16, MXFP4, NVFP4, PAIR_4_8, SharqError, lib, lib_path,
+    ELEM_2_4, F16, F32, BF16, MASK_NONE, MXFP4, NVFP4, PAIR_4_8, PAIR_4_8_GIVEN, SharqError, lib,
+    lib_path,
     sharq_act, sharq_act_bytes, sharq_config, sharq_weight, sharq_weight_bytes, check,
     sharq_act_sizes, sharq_weight_sizes, sharq_status_string, sharq_device_status,
     sharq_prepare, sharq_quantize_weight, sharq_linear, sharq_linear_workspace_size,
@@ -35,17 +36,25 @@ __all__ = [
 
 @dataclass(frozen=True)
 class Config:
+    """fmt, mask and residual mode of sharq_config. residual: True (the method), False, or
+    "unquantized" (ablation: residual against the unquantised backbone). Masks
+    "pair48_given" and "none" are ablations (see include/sharq.h)."""
     fmt: int = NVFP4
     mask: int = PAIR_4_8
-    residual: bool = True
+    residual: bool | str = True
 
     def c(self) -> sharq_config:
-        return sharq_config(self.fmt, self.mask, 1 if self.residual else 0)
+        if self.residual == "unquantized":
+            r = 2
+        else:
+            r = 1 if self.residual else 0
+        return sharq_config(self.fmt, self.mask, r)
 
     @staticmethod
-    def from_names(fmt: str = "nvfp4", mask: str = "pair48", residual: bool = True) -> "Config":
+    def from_names(fmt: str = "nvfp4", mask: str = "pair48", residual: bool | str = True) -> "Config":
         return Config({"nvfp4": NVFP4, "mxfp4": MXFP4}[fmt],
-                      {"pair48": PAIR_4_8, "elem24": ELEM_2_4}[mask], residual)
+                      {"pair48": PAIR_4_8, "elem24": ELEM_2_4, "pair48_given": PAIR_4_8_GIVEN,
+                       "none": MASK_NONE}[mask], residual)
 
 
 def _torch():
@@ -123,7 +132,8 @@ def empty_act(M: int, K: int, cfg: Config, device="cuda") -> PreparedAct:
     torch = _torch()
     sz = sharq_act_bytes()
     check(sharq_act_sizes(M, K, cfg.c(), ctypes.byref(sz)))
-    return PreparedAct(_u8(sz.bq, device), _u8(sz.bs, device), _u8(sz.bm, device),
+    return PreparedAct(_u8(sz.bq, device), _u8(sz.bs, device),
+                       _u8(sz.bm, device) if sz.bm else None,
                        _u8(sz.rq, device) if sz.rq else None,
                        _u8(sz.rs, device) if sz.rs else None,
                        torch.zeros(8, dtype=torch.float32, device=device), M, K, cfg)

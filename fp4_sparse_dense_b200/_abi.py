@@ -8,7 +8,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_PKG, "lib", "libsharq.so")
 
 NVFP4, MXFP4 = 0, 1
-PAIR_4_8, ELEM_2_4 = 0, 1
+PAIR_4_8, ELEM_2_4, PAIR_4_8_GIVEN, MASK_NONE = 0, 1, 2, 3  # the last two: ablations
 F16, BF16, F32 = 0, 1, 2
 
 STATUS = {0: "SHARQ_OK", 1: "SHARQ_ERR_INVALID_ARG", 2: "SHARQ_ERR_UNSUPPORTED",

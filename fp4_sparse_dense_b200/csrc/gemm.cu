@@ -440,7 +440,7 @@ static cudaError_t launch_r(const GemmMaps& m, const GemmParams& p, bool res, bo
 template <int FMT>
 static cudaError_t launch_m(const GemmMaps& m, const GemmParams& p, int mask, bool res, bool f32,
                             int n, cudaStream_t st) {
-  return mask == SHARQ_MASK_PAIR_4_8 ? launch_r<FMT, true>(m, p, res, f32, n, st)
+  return is_pair_mask(mask) ? launch_r<FMT, true>(m, p, res, f32, n, st)
                                      : launch_r<FMT, false>(m, p, res, f32, n, st);
 }
 

@@ -381,7 +381,7 @@ static cudaError_t launch_pair_r(const GemmPairMaps& m, const GemmParams& p, boo
 template <int FMT>
 static cudaError_t launch_pair_m(const GemmPairMaps& m, const GemmParams& p, int mask, bool res,
                                  bool f32, int n, cudaStream_t st) {
-  return mask == SHARQ_MASK_PAIR_4_8 ? launch_pair_r<FMT, true>(m, p, res, f32, n, st)
+  return is_pair_mask(mask) ? launch_pair_r<FMT, true>(m, p, res, f32, n, st)
                                      : launch_pair_r<FMT, false>(m, p, res, f32, n, st);
 }
 

@@ -316,9 +316,14 @@ __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
       uint32_t w[16], L[4];
       unpack16(cur, w);
       if (NORM) rms_apply<BF16>(w, p, row, uint32_t(q) * 256u + uint32_t(wk.u) * 32u);
-      meta = pair_mask(w, s_top2, L, &mx);
+      if (p.mask_given) {  // ablation: the caller's mask stays in bm; only max |x| here
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
+      } else {
+        meta = pair_mask(w, s_top2, L, &mx);
+      }
     }
-    wk.store_meta(q, row, meta);
+    if (!p.mask_given) wk.store_meta(q, row, meta);
 #pragma unroll
     for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
     q = nq;
@@ -393,8 +398,9 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
     if constexpr (NV) decode8_nv(codes, b, tc.s_g, out);
     else decode8<FMT>(codes, b, tc.s_g, out);
   };
+  const bool meta_in = NV || p.mask_given;  // mask read back from bm
   auto load_meta = [&](int it, int r, int q) -> uint32_t {
-    if (!NV || it >= wk.n_items || r >= M) return 0x4444u;
+    if (!meta_in || it >= wk.n_items || r >= M) return 0x4444u;
     return __ldcg(reinterpret_cast<const unsigned short*>(wk.bm + wk.meta_off(q, r)));
   };
 
@@ -418,7 +424,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
       uint32_t w[16], L[4];
       unpack16(cur, w);
       if (NORM) rms_apply<BF16>(w, p, row, k0);
-      if constexpr (NV) {
+      if (meta_in) {
         meta = cmeta;
 #pragma unroll
         for (int g = 0; g < 4; ++g) L[g] = s_nib[(meta >> (4 * g)) & 0xFu];
@@ -433,8 +439,20 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
         x[2 * i] = lo16<BF16>(w[i]);
         x[2 * i + 1] = hi16<BF16>(w[i]);
       }
-      // ---- backbone: one block of 32 logical K
-      const BlockScale bb = scale_of(amax_n<32>(x));
+      // ---- backbone: one block of 32 logical K. With the adaptive mask its max |x| is the
+      // unit's; a supplied mask may drop a group's largest element, so then the max runs
+      // over the kept values only.
+      float a_b;
+      if (p.mask_given) {
+        float xk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          xk[i] = ((L[i >> 3] >> (4 * ((i & 7) >> 1))) & 0xFu) != 4u ? x[i] : 0.f;
+        a_b = amax_n<32>(xk);
+      } else {
+        a_b = amax_n<32>(x);
+      }
+      const BlockScale bb = scale_of(a_b);
       bsf = bb.code;
       uint32_t c[4];
 #pragma unroll
@@ -452,7 +470,13 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           float d[8];
-          decode_of(__byte_perm(c[g], 0u, L[g]), bb, d);
+          if (p.res_unquant) {  // ablation: against the unquantised backbone
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              d[j] = ((L[g] >> (4 * (j >> 1))) & 0xFu) != 4u ? x[8 * g + j] : 0.f;
+          } else {
+            decode_of(__byte_perm(c[g], 0u, L[g]), bb, d);
+          }
 #pragma unroll
           for (int j = 0; j < 8; j += 2) {
             const float2 t = sub2_rn(make_float2(x[8 * g + j], x[8 * g + j + 1]),
@@ -508,7 +532,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
         }
       }
     }
-    if constexpr (!NV) wk.store_meta(q, row, meta);
+    if (!meta_in) wk.store_meta(q, row, meta);
 #pragma unroll
     for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
     cmeta = nmeta;
@@ -597,8 +621,9 @@ __global__ void __launch_bounds__(256) prep_elem_kernel(PrepParams p) {
         }
         const int c01 = key[0] > key[1], c02 = key[0] > key[2], c03 = key[0] > key[3];
         const int c12 = key[1] > key[2], c13 = key[1] > key[3], c23 = key[2] > key[3];
-        const bool kp[4] = {(3 - c01 - c02 - c03) < 2, (c01 + 2 - c12 - c13) < 2,
-                            (c02 + c12 + 1 - c23) < 2, (c03 + c13 + c23) < 2};
+        const bool all = p.keep_all != 0;  // ablation: no mask, plain FP4 of x
+        const bool kp[4] = {all || (3 - c01 - c02 - c03) < 2, all || (c01 + 2 - c12 - c13) < 2,
+                            all || (c02 + c12 + 1 - c23) < 2, all || (c03 + c13 + c23) < 2};
         const int i0 = kp[0] ? 0 : (kp[1] ? 1 : 2);
         const int i1 = kp[3] ? 3 : (kp[2] ? 2 : 1);
         meta |= uint32_t(i0 | (i1 << 2)) << (4 * g);
@@ -621,11 +646,14 @@ __global__ void __launch_bounds__(256) prep_elem_kernel(PrepParams p) {
       }
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.bq) + size_t(r) * (K / 2) + k0 / 2) =
           make_uint4(bcodes[0], bcodes[1], bcodes[2], bcodes[3]);
-      *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.bm) + size_t(r) * (K / 8) + k0 / 8) =
-          meta;
+      if (!p.keep_all)
+        *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.bm) + size_t(r) * (K / 8) + k0 / 8) =
+            meta;
       if (RESIDUAL) {
+        // ablation res_unquant: against the unquantised backbone (x - x = +0 where kept)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r_val[i] = (kept >> i) & 1u ? __fsub_rn(x[i], deq[i]) : x[i];
+        for (int i = 0; i < 32; ++i)
+          r_val[i] = (kept >> i) & 1u ? __fsub_rn(x[i], p.res_unquant ? x[i] : deq[i]) : x[i];
       }
     }
 
@@ -688,7 +716,7 @@ static cudaError_t launch_pdl(void (*kern)(Args...), unsigned blocks, cudaStream
 
 template <bool BF16, int FMT, bool RES, bool NORM>
 static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
-  if (mask == SHARQ_MASK_PAIR_4_8) {
+  if (is_pair_mask(mask)) {
     auto kern = prep_pair_kernel<BF16, FMT, RES, NORM>;
     static int per_sm = 0;  // resident CTAs per SM (one value per instantiation)
     if (per_sm == 0) {

@@ -91,7 +91,7 @@ static cudaError_t launch_wq_t(const WeightQuantParams& p, cudaStream_t st) {
 
 template <bool BF16>
 static cudaError_t launch_wq_b(const WeightQuantParams& p, int fmt, int mask, cudaStream_t st) {
-  const bool pair = mask == SHARQ_MASK_PAIR_4_8;
+  const bool pair = is_pair_mask(mask);
   if (fmt == SHARQ_NVFP4)
     return pair ? launch_wq_t<BF16, SHARQ_NVFP4, 32, true>(p, st)
                 : launch_wq_t<BF16, SHARQ_NVFP4, 16, false>(p, st);

@@ -60,8 +60,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 sharq_status check_cfg(sharq_config c) {
   if (c.fmt != SHARQ_NVFP4 && c.fmt != SHARQ_MXFP4) return SHARQ_ERR_INVALID_ARG;
-  if (c.mask != SHARQ_MASK_PAIR_4_8 && c.mask != SHARQ_MASK_ELEM_2_4) return SHARQ_ERR_INVALID_ARG;
-  if (c.residual != 0 && c.residual != 1) return SHARQ_ERR_INVALID_ARG;
+  if (c.mask < SHARQ_MASK_PAIR_4_8 || c.mask > SHARQ_MASK_NONE) return SHARQ_ERR_INVALID_ARG;
+  if (c.residual < 0 || c.residual > 2) return SHARQ_ERR_INVALID_ARG;
   return SHARQ_OK;
 }
 
@@ -193,11 +193,11 @@ sharq_status act_sizes(int32_t M, int32_t K, sharq_config c, sharq_act_bytes* o)
   if (!o || M < 1 || K < 256 || K % 256 != 0) return SHARQ_ERR_INVALID_ARG;
   sharq_status s = check_cfg(c);
   if (s != SHARQ_OK) return s;
-  const bool pair = c.mask == SHARQ_MASK_PAIR_4_8;
+  const bool pair = is_pair_mask(c.mask);
   const size_t m = size_t(M), k = size_t(K);
   o->bq = pair ? m * k / 4 : m * k / 2;
   o->bs = tiled_bytes(m, k / size_t(backbone_block(c.fmt, c.mask)));
-  o->bm = pair ? round_up(m, 128) * k / 16 : m * k / 8;
+  o->bm = pair ? round_up(m, 128) * k / 16 : (c.mask == SHARQ_MASK_NONE ? 0 : m * k / 8);
   o->rq = c.residual ? m * k / 2 : 0;
   o->rs = c.residual ? tiled_bytes(m, k / size_t(residual_block(c.fmt))) : 0;
   return SHARQ_OK;
@@ -210,7 +210,7 @@ sharq_status weight_sizes(int32_t K, int32_t N, sharq_config c, sharq_weight_byt
   const size_t k = size_t(K), n = size_t(N);
   o->codes = n * k / 2;
   o->scales_dense = tiled_bytes(n, k / size_t(dense_view_block(c.fmt)));
-  o->scales_sparse = c.mask == SHARQ_MASK_PAIR_4_8 ? tiled_bytes(n, k / 32) : 0;
+  o->scales_sparse = is_pair_mask(c.mask) ? tiled_bytes(n, k / 32) : 0;
   return SHARQ_OK;
 }
 
@@ -230,13 +230,13 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
   sharq_act_bytes sz;
   sharq_status s = act_sizes(a->M, a->K, a->cfg, &sz);
   if (s != SHARQ_OK) return s;
-  const bool res = a->cfg.residual == 1;
+  const bool res = a->cfg.residual != 0;
   const bool norm = gamma != nullptr;
-  if (norm && a->cfg.mask != SHARQ_MASK_PAIR_4_8) return SHARQ_ERR_UNSUPPORTED;
+  const bool pair = is_pair_mask(a->cfg.mask), none = a->cfg.mask == SHARQ_MASK_NONE;
+  if (norm && !pair) return SHARQ_ERR_UNSUPPORTED;
   // the pair-mask kernels address X and their outputs with 32-bit offsets
-  if (a->cfg.mask == SHARQ_MASK_PAIR_4_8 && size_t(a->M) * size_t(a->K) >= (size_t(1) << 31))
-    return SHARQ_ERR_UNSUPPORTED;
-  if (!a->bq || !a->bs || !a->bm || !a->tensor_scale || (res && (!a->rq || !a->rs)) ||
+  if (pair && size_t(a->M) * size_t(a->K) >= (size_t(1) << 31)) return SHARQ_ERR_UNSUPPORTED;
+  if (!a->bq || !a->bs || (!a->bm && !none) || !a->tensor_scale || (res && (!a->rq || !a->rs)) ||
       (norm && !rstd))
     return SHARQ_ERR_INVALID_ARG;
   if (norm && !(eps >= 0.f && eps < 1e30f)) return SHARQ_ERR_INVALID_ARG;
@@ -251,7 +251,7 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
   // the pair-mask kernels reduce the NVFP4 tensor amax themselves (state in
   // tensor_scale[2..3]); the element-mask kernel takes it from a separate pass into
   // tensor_scale[1]
-  if (a->cfg.fmt == SHARQ_NVFP4 && a->cfg.mask == SHARQ_MASK_ELEM_2_4) {
+  if (a->cfg.fmt == SHARQ_NVFP4 && !pair) {
     if (cudaMemsetAsync(a->tensor_scale + 1, 0, sizeof(float), st) != cudaSuccess)
       return SHARQ_ERR_CUDA;
     s = from_cuda(launch_amax(X, bf16, size_t(a->M) * size_t(a->K),
@@ -275,6 +275,9 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
   p.gamma = gamma;
   p.rstd = rstd;
   p.eps = eps;
+  p.mask_given = a->cfg.mask == SHARQ_MASK_PAIR_4_8_GIVEN;
+  p.keep_all = none;
+  p.res_unquant = a->cfg.residual == 2;
   return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
 }
 }  // namespace
@@ -310,7 +313,7 @@ sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, const sharq
   sharq_weight_bytes sz;
   sharq_status s = weight_sizes(w->K, w->N, w->cfg, &sz);
   if (s != SHARQ_OK) return s;
-  const bool pair = w->cfg.mask == SHARQ_MASK_PAIR_4_8;
+  const bool pair = is_pair_mask(w->cfg.mask);
   if (!w->codes || !w->scales_dense || !w->tensor_scale || (pair && !w->scales_sparse))
     return SHARQ_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(w->codes) || !aligned16(w->scales_dense) ||
@@ -374,7 +377,7 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   sharq_status s = act_sizes(a->M, a->K, a->cfg, &asz);
   if (s != SHARQ_OK) return s;
   if ((s = weight_sizes(w->K, w->N, w->cfg, &wsz)) != SHARQ_OK) return s;
-  const bool res = a->cfg.residual == 1, pair = a->cfg.mask == SHARQ_MASK_PAIR_4_8;
+  const bool res = a->cfg.residual != 0, pair = is_pair_mask(a->cfg.mask);
   if (!a->bq || !a->bs || !a->tensor_scale || (pair && !a->bm) || (res && (!a->rq || !a->rs)) ||
       !w->codes || !w->tensor_scale || ((res || !pair) && !w->scales_dense) ||
       (pair && !w->scales_sparse))

@@ -25,6 +25,10 @@ struct PrepParams {
   const void* gamma;    // [K] 16-bit, same dtype as X
   float* rstd;          // [M] per-row 1 / sqrt(mean x^2 + eps), written by rms_kernel
   float eps;
+  // ablation modes (runtime flags: not on the method's path)
+  int mask_given;       // pair mask read from bm instead of chosen per row
+  int keep_all;         // no mask: every element on the (dense) backbone
+  int res_unquant;      // residual against the unquantised backbone
 };
 
 struct WeightQuantParams {
@@ -76,14 +80,19 @@ struct GemmPairMaps {
 cudaError_t launch_gemm_pair(const GemmPairMaps& maps, const GemmParams& p, int fmt, int mask,
                              bool residual, bool out_f32, int num_sms, cudaStream_t st);
 
+// masks whose backbone is stored compressed and runs through the sparse MMA
+inline bool is_pair_mask(int mask) {
+  return mask == SHARQ_MASK_PAIR_4_8 || mask == SHARQ_MASK_PAIR_4_8_GIVEN;
+}
+
 // block sizes along K
 inline int residual_block(int fmt) { return fmt == SHARQ_NVFP4 ? 16 : 32; }
 inline int backbone_block(int fmt, int mask) {
-  return mask == SHARQ_MASK_PAIR_4_8 ? 32 : residual_block(fmt);
+  return is_pair_mask(mask) ? 32 : residual_block(fmt);
 }
 inline int weight_block(int fmt, int mask) {
   if (fmt == SHARQ_MXFP4) return 32;
-  return mask == SHARQ_MASK_PAIR_4_8 ? 32 : 16;
+  return is_pair_mask(mask) ? 32 : 16;
 }
 inline int dense_view_block(int fmt) { return fmt == SHARQ_NVFP4 ? 16 : 32; }
 

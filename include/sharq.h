@@ -60,20 +60,36 @@ typedef enum { SHARQ_NVFP4 = 0, SHARQ_MXFP4 = 1 } sharq_format;
  * (max |x|, then min |x|), ties to the lower pair. ELEM_2_4: in every 4 keep the 2 largest
  * |x|, ties to the lower index; the backbone is then stored zero-filled and runs through
  * the dense MMA (sm_100a has no element-wise 2:4 pattern for block-scaled FP4). */
-typedef enum { SHARQ_MASK_PAIR_4_8 = 0, SHARQ_MASK_ELEM_2_4 = 1 } sharq_mask;
+typedef enum {
+  SHARQ_MASK_PAIR_4_8 = 0,
+  SHARQ_MASK_ELEM_2_4 = 1,
+  /* Ablation modes (the page's referee asks for them; not part of the method):
+   * PAIR_4_8_GIVEN: the pair-wise 4:8 mask is not chosen per row but read from act->bm,
+   * which the caller fills in the PAIR metadata layout before sharq_prepare (a static
+   * mask: one channel set for the whole tensor, e.g. from calibration statistics); the
+   * rest is PAIR_4_8. NONE: no mask, every element is on the "backbone", i.e. plain FP4
+   * of x in the residual's block size through the dense MMA (with residual on, a second
+   * dense FP4 term r = x - deq(Q(x))). */
+  SHARQ_MASK_PAIR_4_8_GIVEN = 2,
+  SHARQ_MASK_NONE = 3
+} sharq_mask;
 
 typedef enum { SHARQ_F16 = 0, SHARQ_BF16 = 1, SHARQ_F32 = 2 } sharq_dtype;
 
 typedef struct {
   int32_t fmt;      /* sharq_format */
   int32_t mask;     /* sharq_mask */
-  int32_t residual; /* 1: backbone + residual (the method); 0: backbone only */
+  int32_t residual; /* 1: backbone + residual (the method); 0: backbone only;
+                       2: ablation, residual against the unquantised backbone
+                       (r = x - backbone: 0 where the mask keeps, x elsewhere) */
 } sharq_config;
 
 /* Block sizes along K (logical positions per scale), fixed by the MMA consuming them:
  *   residual:  16 (NVFP4) | 32 (MXFP4)
  *   backbone:  32 for PAIR_4_8 (16 kept values); the residual's size for ELEM_2_4
- *   weight:    32 for PAIR_4_8 or MXFP4; 16 for NVFP4 + ELEM_2_4
+ *   weight:    32 for PAIR_4_8(_GIVEN) or MXFP4; 16 for NVFP4 + ELEM_2_4 / NONE
+ *   (PAIR_4_8_GIVEN has the sizes and layouts of PAIR_4_8; NONE those of ELEM_2_4,
+ *   without metadata: act->bm is unused and may be NULL)
  *
  * Byte layouts (all row-major in the sense given):
  *   FP4 codes:  two per byte, even K index in the low nibble, rows K-major.

@@ -26,7 +26,9 @@ def cfg_of(fmt: str, mask: str, residual: bool = True):
 
 def act_bytes(act) -> dict:
     out = {"tensor_scale": act.tensor_scale[:1].cpu().numpy(),
-           "bq": act.bq.cpu().numpy(), "bs": act.bs.cpu().numpy(), "bm": act.bm.cpu().numpy()}
+           "bq": act.bq.cpu().numpy(), "bs": act.bs.cpu().numpy()}
+    if act.bm is not None:
+        out["bm"] = act.bm.cpu().numpy()
     if act.rq is not None:
         out["rq"] = act.rq.cpu().numpy()
         out["rs"] = act.rs.cpu().numpy()

@@ -54,25 +54,29 @@ def test_status_strings(sq):
     assert sq.sharq_status_string(99) == b"SHARQ_ERR_UNKNOWN"
 
 
-CFGS = [(f, m, r) for f in ("nvfp4", "mxfp4") for m in ("pair48", "elem24") for r in (True, False)]
+CFGS = [(f, m, r) for f in ("nvfp4", "mxfp4") for m in ("pair48", "elem24", "pair48_given", "none")
+        for r in (True, False)]
 
 
 @pytest.mark.parametrize("fmt,mask,res", CFGS)
 @pytest.mark.parametrize("M,K", [(1, 256), (16, 256), (130, 512), (300, 4096)])
 def test_act_sizes_match_oracle_layouts(sq, fmt, mask, res, M, K):
     x = np.random.default_rng(0).standard_normal((M, K)).astype(np.float32)
-    want = S.act_buffers(S.prepare(x, fmt, mask, residual=res))
+    given = S.keep_pairs48(x) if mask == "pair48_given" else None
+    want = S.act_buffers(S.prepare(x, fmt, mask, residual=res, given=given))
     sz = sq.sharq_act_bytes()
     cfg = sq.Config.from_names(fmt, mask, res).c()
     assert sq.sharq_act_sizes(M, K, cfg, ctypes.byref(sz)) == 0
-    assert sz.bq == want["bq"].size and sz.bs == want["bs"].size and sz.bm == want["bm"].size
+    assert sz.bq == want["bq"].size and sz.bs == want["bs"].size
+    assert sz.bm == (want["bm"].size if "bm" in want else 0)
     if res:
         assert sz.rq == want["rq"].size and sz.rs == want["rs"].size
     else:
         assert sz.rq == 0 and sz.rs == 0
 
 
-@pytest.mark.parametrize("fmt,mask", [(f, m) for f in ("nvfp4", "mxfp4") for m in ("pair48", "elem24")])
+@pytest.mark.parametrize("fmt,mask", [(f, m) for f in ("nvfp4", "mxfp4")
+                                      for m in ("pair48", "elem24", "pair48_given", "none")])
 def test_weight_sizes_match_oracle_layouts(sq, fmt, mask):
     K, N = 512, 384
     w = np.random.default_rng(1).standard_normal((K, N)).astype(np.float32)
@@ -80,7 +84,7 @@ def test_weight_sizes_match_oracle_layouts(sq, fmt, mask):
     sz = sq.sharq_weight_bytes()
     assert sq.sharq_weight_sizes(K, N, sq.Config.from_names(fmt, mask).c(), ctypes.byref(sz)) == 0
     assert sz.codes == want["codes"].size and sz.scales_dense == want["scales_dense"].size
-    assert sz.scales_sparse == (want["scales_sparse"].size if mask == "pair48" else 0)
+    assert sz.scales_sparse == (want["scales_sparse"].size if S.is_pair(mask) else 0)
 
 
 def test_bad_shapes_and_configs_rejected(sq):
@@ -89,7 +93,8 @@ def test_bad_shapes_and_configs_rejected(sq):
     assert sq.sharq_act_sizes(16, 200, ok, ctypes.byref(sz)) == 1   # K % 256
     assert sq.sharq_act_sizes(0, 256, ok, ctypes.byref(sz)) == 1    # M < 1
     assert sq.sharq_act_sizes(16, 256, sq.sharq_config(7, 0, 1), ctypes.byref(sz)) == 1
-    assert sq.sharq_act_sizes(16, 256, sq.sharq_config(0, 0, 2), ctypes.byref(sz)) == 1
+    assert sq.sharq_act_sizes(16, 256, sq.sharq_config(0, 0, 3), ctypes.byref(sz)) == 1
+    assert sq.sharq_act_sizes(16, 256, sq.sharq_config(0, 4, 1), ctypes.byref(sz)) == 1
     wz = sq.sharq_weight_bytes()
     assert sq.sharq_weight_sizes(256, 100, ok, ctypes.byref(wz)) == 1  # N % 128
 
