@@ -31,8 +31,32 @@ sys.path.insert(0, ROOT)
 
 METRIC = "SharQ linear TFLOPS (2MNK/t) and % FP4 peak; prep kernel HBM GB/s"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
-PREP_BYTES_PER_ELEM = {"pair48": 2 + 0.25 + 0.0625 + 0.0625 + 0.5 + 0.0625,
-                       "elem24": 2 + 0.5 + 0.0625 + 0.125 + 0.5 + 0.0625}
+
+
+def prep_bytes_per_elem(fmt: str, mask: str, residual: bool) -> float:
+    """Algorithmic HBM bytes per X element of the preparation: the 16-bit read plus every
+    output (codes, scales, metadata); the pair-wise backbone is stored compressed."""
+    rb = 16 if fmt == "nvfp4" else 32
+    pair = mask.startswith("pair48")
+    b = 2.0 + (0.25 if pair else 0.5) + 1.0 / (32 if pair else rb)
+    b += {"pair48": 1 / 16, "pair48_given": 0.0, "elem24": 1 / 8, "none": 0.0}[mask]
+    if residual:
+        b += 0.5 + 1.0 / rb
+    return b
+
+
+def metric_ceiling(mask: str, residual: bool) -> float:
+    """2MNK / t at full tensor-pipe use, as a fraction of the dense FP4 peak: the sparse MMA
+    runs the backbone's 2MNK at twice the dense rate, the dense MMAs at the dense rate."""
+    t = (0.5 if mask.startswith("pair48") else 1.0) + (1.0 if residual else 0.0)
+    return 1.0 / t
+
+
+def prep_kernels(fmt: str, mask: str) -> list:
+    if mask.startswith("pair48"):
+        return (["prep_mask_kernel"] if fmt == "nvfp4" else []) + ["prep_pair_kernel"]
+    return (["amax_kernel"] if fmt == "nvfp4" else []) + ["prep_elem_kernel"]
+
 
 WORKLOADS = {
     # name: (M, K, N, per_row_outliers)
@@ -156,18 +180,31 @@ def make_inputs(workload: str, seed: int):
     return x, w
 
 
-def cpu_baseline(workload: str, budget_s: float, x, qw):
+def oracle_modes(args) -> dict:
+    """prepare() keyword arguments of the oracle for the bench's --fmt/--mask/--residual."""
+    kw = {"fmt": args.fmt, "mask": args.mask, "residual": args.residual != "off"}
+    if args.residual == "unquantized":
+        kw["residual_ref"] = "unquantized"
+    return kw
+
+
+def cpu_baseline(workload: str, budget_s: float, x, qw, kw=None):
     """The oracle as it stands, on a bounded sample: blocks of 16 token rows prepared and
     multiplied by the whole weight (quantised beforehand: an offline step) until the
     budget of CPU time is used. Returns (TFLOP/s, cores, sample description)."""
     from oracle import sharq as S
+    kw = dict(kw or {})
     M, K, N, _ = WORKLOADS[workload]
-    amax = S.amax_of(x.values)
+    amax = S.amax_of(x.values) if kw.get("fmt", "nvfp4") == "nvfp4" else None
+    given = None
+    if kw.get("mask") == S.PAIR48_GIVEN:
+        given = S.static_keep_pairs48(x.values, 16)
     rows = 16
     t_used, n_rows = 0.0, 0
     while t_used < budget_s and n_rows < M:
         t0 = time.perf_counter()
-        p = S.prepare(x.values[n_rows:n_rows + rows], amax=amax)
+        xs = x.values[n_rows:n_rows + rows]
+        p = S.prepare(xs, amax=amax, given=None if given is None else given[: len(xs)], **kw)
         S.linear(p, qw)
         t_used += time.perf_counter() - t0
         n_rows += rows
@@ -184,13 +221,14 @@ def run_reference(args):
     from oracle import sharq as S
     M, K, N, _ = WORKLOADS[args.workload]
     x, w = make_inputs(args.workload, rank_seed(0))
-    qw = S.quantize_weight(w.values)  # offline step, outside the timed samples
+    kw = oracle_modes(args)
+    qw = S.quantize_weight(w.values, args.fmt, args.mask)  # offline, outside the samples
     budget = max(1.0, 90.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_baseline(args.workload, budget, x, qw)
+        cpu_baseline(args.workload, budget, x, qw, kw)
     vals = []
     for _ in range(args.steps):
-        v, cores, sample = cpu_baseline(args.workload, budget, x, qw)
+        v, cores, sample = cpu_baseline(args.workload, budget, x, qw, kw)
         vals.append(v)
     value = float(np.mean(vals))
     line = {
@@ -198,8 +236,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 2.0 * M * N * K / (value * 1e12) * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": "nvfp4",
-                   "mask": "pair48"},
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": args.fmt,
+                   "mask": args.mask, "residual": args.residual},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -223,16 +261,30 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     dev = torch.device("cuda", local)
     M, K, N, _ = WORKLOADS[args.workload]
-    cfg = sq.Config()  # NVFP4, pair-wise 4:8, residual on
+    res_mode = {"on": True, "off": False, "unquantized": "unquantized"}[args.residual]
+    cfg = sq.Config.from_names(args.fmt, args.mask, res_mode)  # default: the method
+    has_res = args.residual != "off"
 
     x16, w16 = make_inputs(args.workload, rank_seed(rank))
     from tests.gpu_helpers import to_device
     n_sets = 3
     X = [to_device(x16).to(dev) for _ in range(n_sets)]
     W = [to_device(w16).to(dev) for _ in range(2)]
-    QW = [sq.quantize_weight(w) for w in W]
+    QW = [sq.quantize_weight(w, cfg) for w in W]
     ACT = [sq.empty_act(M, K, cfg, dev) for _ in range(n_sets)]
     Y = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(n_sets)]
+    if args.mask == "pair48_given":
+        # ablation set-up (outside the timed region): a static mask, the pair mask of the
+        # per-column max |x| of the first input set, replicated to every row in the PAIR
+        # metadata layout ([K/256 slices][rows padded to 128][16 bytes], padding 0x44)
+        col = X[0].abs().amax(dim=0, keepdim=True).to(X[0].dtype)
+        one = sq.prepare(col, sq.Config.from_names(args.fmt, "pair48", False))
+        KS, Mp = K // 256, (M + 127) // 128 * 128
+        row0 = one.bm.view(KS, 128, 16)[:, :1, :]
+        full = torch.full((KS, Mp, 16), 0x44, dtype=torch.uint8, device=dev)
+        full[:, :M, :] = row0
+        for a in ACT:
+            a.bm[: full.numel()].copy_(full.view(-1))
     WS = sq.linear_workspace(M, N, K, cfg, dev)  # split-K scratch (None for prefill shapes)
     stream = torch.cuda.current_stream()
 
@@ -307,15 +359,16 @@ def run_gpu(args):
         gemm_avg = float(np.mean(gemm_ms))
         prep_avg = float(np.mean(prep_ms))
         gemm_tflops = flops / (gemm_avg * 1e-3) / 1e12
-        prep_gbs = M * K * PREP_BYTES_PER_ELEM["pair48"] / (prep_avg * 1e-3) / 1e9
+        bpe = prep_bytes_per_elem(args.fmt, args.mask, has_res)
+        prep_gbs = M * K * bpe / (prep_avg * 1e-3) / 1e9
         traffic = traffic_from_profile(args.workload)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
             "data": "synthetic",
-            "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": "nvfp4",
-                       "mask": "pair48", "residual": True, "out": "bf16",
+            "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": args.fmt,
+                       "mask": args.mask, "residual": args.residual, "out": "bf16",
                        "l2": f"{n_sets} rotating input sets (> 126 MB L2 per step)",
                        "parallelism": f"dp{world}"},
             "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
@@ -323,12 +376,12 @@ def run_gpu(args):
                          "traffic": traffic,
                          "peak_source": f"{peak_src}: bf16 sustained {bf16_sus} x "
                                         f"{FP4_OVER_BF16} (nominal FP4:BF16)",
-                         "ceiling_frac": 2.0 / 3.0,
+                         "ceiling_frac": metric_ceiling(args.mask, has_res),
                          "kernel": gemm_kernel_name(M, N), "kernel_ms": gemm_avg},
             "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
                      "frac": prep_gbs / hbm,
-                     "bytes_per_elem": PREP_BYTES_PER_ELEM["pair48"],
-                     "kernel": "prep_mask_kernel + prep_pair_kernel",
+                     "bytes_per_elem": bpe,
+                     "kernel": " + ".join(prep_kernels(args.fmt, args.mask)),
                      "note": "two launches (mask, metadata and tensor amax; then quantisation, "
                              "started early by programmatic dependent launch); algorithmic "
                              "bytes count X once"},
@@ -336,13 +389,15 @@ def run_gpu(args):
             "pct_fp4_peak": 100.0 * gemm_tflops / fp4_peak,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
                     "d2h_bytes_per_step": M * N * 2},
-            "gpu_launches": (2 + 1 + (1 if WS is not None else 0)) * args.steps,
+            "gpu_launches": (len(prep_kernels(args.fmt, args.mask)) + 1 +
+                             (1 if WS is not None else 0)) * args.steps,
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline and world == 1:
             from oracle import sharq as S
-            qw_cpu = S.quantize_weight(w16.values)
-            v, cores, sample = cpu_baseline(args.workload, args.cpu_budget, x16, qw_cpu)
+            qw_cpu = S.quantize_weight(w16.values, args.fmt, args.mask)
+            v, cores, sample = cpu_baseline(args.workload, args.cpu_budget, x16, qw_cpu,
+                                            oracle_modes(args))
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores,
                                     "kind": "oracle", "sample": sample}
         print(json.dumps(line), flush=True)
@@ -360,6 +415,12 @@ def main():
     ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
     ap.add_argument("--workload", default="mlp_gate_up", choices=list(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
+    ap.add_argument("--mask", default="pair48",
+                    choices=["pair48", "elem24", "pair48_given", "none"],
+                    help="pair48 is the method; the others are ablations / baselines "
+                         "(none with --residual off: plain FP4)")
+    ap.add_argument("--residual", default="on", choices=["on", "off", "unquantized"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
