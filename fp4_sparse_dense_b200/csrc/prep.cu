@@ -291,8 +291,9 @@ __device__ __forceinline__ void unpack16(const uint4* c, uint32_t* w) {
 // First NVFP4 preparation kernel (pair mask): streams X from HBM, computes the mask, writes
 // the metadata (padding rows included) and folds max |x| into the tensor amax. Its integer
 // work hides under the HBM reads.
-template <bool BF16, bool NORM>
+template <bool BF16, bool NORM, bool ABL>
 __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
+  const bool mask_given = ABL && p.mask_given;  // ablation flags compile away unless ABL
   // the quantisation kernel may start its prologue now; it waits for this grid's completion
   // (griddepcontrol.wait) before it reads anything written here
   ptx::griddep_launch_dependents();
@@ -316,14 +317,14 @@ __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
       uint32_t w[16], L[4];
       unpack16(cur, w);
       if (NORM) rms_apply<BF16>(w, p, row, uint32_t(q) * 256u + uint32_t(wk.u) * 32u);
-      if (p.mask_given) {  // ablation: the caller's mask stays in bm; only max |x| here
+      if (mask_given) {  // ablation: the caller's mask stays in bm; only max |x| here
 #pragma unroll
         for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, w[i] & 0x7FFF7FFFu);
       } else {
         meta = pair_mask(w, s_top2, L, &mx);
       }
     }
-    if (!p.mask_given) wk.store_meta(q, row, meta);
+    if (!mask_given) wk.store_meta(q, row, meta);
 #pragma unroll
     for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
     q = nq;
@@ -347,9 +348,11 @@ __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
 // which is kept); byte permutes then keep the kept pairs' code bytes, either compressed
 // (the backbone operand) or in place with zeros elsewhere, which dequantise to the backbone
 // at kept positions and +0 elsewhere, so r = x - deq needs no per-element selection.
-template <bool BF16, int FMT, bool RESIDUAL, bool NORM>
+template <bool BF16, int FMT, bool RESIDUAL, bool NORM, bool ABL>
 __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   constexpr bool NV = FMT == SHARQ_NVFP4;
+  // ablation flags compile away unless ABL (the method's instantiation stays lean)
+  const bool mask_given = ABL && p.mask_given, res_unquant = ABL && p.res_unquant;
   constexpr int RB = NV ? 16 : 32;  // residual block
   __shared__ uint32_t s_top2[64];
   __shared__ uint32_t s_nib[16];
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
     if constexpr (NV) decode8_nv(codes, b, tc.s_g, out);
     else decode8<FMT>(codes, b, tc.s_g, out);
   };
-  const bool meta_in = NV || p.mask_given;  // mask read back from bm
+  const bool meta_in = NV || mask_given;  // mask read back from bm
   auto load_meta = [&](int it, int r, int q) -> uint32_t {
     if (!meta_in || it >= wk.n_items || r >= M) return 0x4444u;
     return __ldcg(reinterpret_cast<const unsigned short*>(wk.bm + wk.meta_off(q, r)));
@@ -443,7 +446,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
       // unit's; a supplied mask may drop a group's largest element, so then the max runs
       // over the kept values only.
       float a_b;
-      if (p.mask_given) {
+      if (mask_given) {
         float xk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i)
@@ -470,7 +473,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           float d[8];
-          if (p.res_unquant) {  // ablation: against the unquantised backbone
+          if (res_unquant) {  // ablation: against the unquantised backbone
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               d[j] = ((L[g] >> (4 * (j >> 1))) & 0xFu) != 4u ? x[8 * g + j] : 0.f;
@@ -714,20 +717,26 @@ static cudaError_t launch_pdl(void (*kern)(Args...), unsigned blocks, cudaStream
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <bool BF16, int FMT, bool RES, bool NORM>
+// CTAs of a persistent preparation kernel: enough warp items for every warp, at most what
+// fits on the GPU at once (resident CTAs per SM from the occupancy calculator, cached)
+template <typename Kern>
+static cudaError_t persistent_blocks(Kern kern, int* per_sm, const PrepParams& p, int num_sms,
+                                     unsigned* blocks) {
+  if (*per_sm == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, 256, 0);
+    if (e != cudaSuccess) return e;
+    if (*per_sm < 1) *per_sm = 1;
+  }
+  const long items = long(p.Mp / 4) * (p.K / 256);
+  long b = (items + 7) / 8;
+  const long cap = long(num_sms) * *per_sm;
+  *blocks = unsigned(b < cap ? b : cap);
+  return cudaSuccess;
+}
+
+template <bool BF16, int FMT, bool RES, bool NORM, bool ABL>
 static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
   if (is_pair_mask(mask)) {
-    auto kern = prep_pair_kernel<BF16, FMT, RES, NORM>;
-    static int per_sm = 0;  // resident CTAs per SM (one value per instantiation)
-    if (per_sm == 0) {
-      cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
-      if (e != cudaSuccess) return e;
-      if (per_sm < 1) per_sm = 1;
-    }
-    const long items = long(p.Mp / 4) * (p.K / 256);
-    long blocks = (items + 7) / 8;
-    const long cap = long(num_sms) * per_sm;
-    if (blocks > cap) blocks = cap;
     cudaError_t e = cudaSuccess;
     if (NORM) {  // per-row rstd first: one warp per row
       long rb = (long(p.M) + 7) / 8;
@@ -736,10 +745,17 @@ static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cud
       if (e != cudaSuccess) return e;
     }
     if (FMT == SHARQ_NVFP4) {
-      e = launch_pdl(prep_mask_kernel<BF16, NORM>, unsigned(blocks), st, p);
-      if (e != cudaSuccess) return e;
+      auto mk = prep_mask_kernel<BF16, NORM, ABL>;
+      static int mk_per_sm = 0;
+      unsigned mb = 0;
+      if ((e = persistent_blocks(mk, &mk_per_sm, p, num_sms, &mb)) != cudaSuccess) return e;
+      if ((e = launch_pdl(mk, mb, st, p)) != cudaSuccess) return e;
     }
-    e = launch_pdl(kern, unsigned(blocks), st, p);
+    auto kern = prep_pair_kernel<BF16, FMT, RES, NORM, ABL>;
+    static int per_sm = 0;
+    unsigned blocks = 0;
+    if ((e = persistent_blocks(kern, &per_sm, p, num_sms, &blocks)) != cudaSuccess) return e;
+    e = launch_pdl(kern, blocks, st, p);
     if (e != cudaSuccess) return e;
   } else {
     if (NORM) return cudaErrorNotSupported;
@@ -749,10 +765,17 @@ static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cud
   return cudaGetLastError();
 }
 
+template <bool BF16, int FMT, bool RES, bool NORM>
+static cudaError_t launch_prep_a(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
+  const bool abl = p.mask_given || p.res_unquant;
+  return abl ? launch_prep_t<BF16, FMT, RES, NORM, true>(p, mask, num_sms, st)
+             : launch_prep_t<BF16, FMT, RES, NORM, false>(p, mask, num_sms, st);
+}
+
 template <bool BF16, int FMT, bool RES>
 static cudaError_t launch_prep_n(const PrepParams& p, int mask, bool norm, int n, cudaStream_t st) {
-  return norm ? launch_prep_t<BF16, FMT, RES, true>(p, mask, n, st)
-              : launch_prep_t<BF16, FMT, RES, false>(p, mask, n, st);
+  return norm ? launch_prep_a<BF16, FMT, RES, true>(p, mask, n, st)
+              : launch_prep_a<BF16, FMT, RES, false>(p, mask, n, st);
 }
 
 template <bool BF16, int FMT>
