@@ -21,7 +21,7 @@ from ._abi import (  # noqa: F401
     sharq_act, sharq_act_bytes, sharq_config, sharq_weight, sharq_weight_bytes, check,
     sharq_act_sizes, sharq_weight_sizes, sharq_status_string, sharq_device_status,
     sharq_prepare, sharq_quantize_weight, sharq_linear, sharq_linear_workspace_size,
-    sharq_linear_noalloc, sharq_prepare_rmsnorm,
+    sharq_linear_noalloc, sharq_prepare_rmsnorm, sharq_wait_probe,
 )
 
 __all__ = [

@@ -283,6 +283,30 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
 }  // namespace
 }  // namespace sharq
 
+namespace sharq {
+namespace {
+// One thread waits for *flag == expected with the same bounded-wait discipline as the
+// GEMM's pipeline waits; on expiry the status word gets SHARQ_ERR_TIMEOUT.
+__global__ void wait_probe_kernel(const uint32_t* flag, uint32_t expected, uint64_t limit_ns,
+                                  unsigned int* status) {
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (uint32_t it = 0;; ++it) {
+    if (*reinterpret_cast<const volatile uint32_t*>(flag) == expected) return;
+    if ((it & 63u) == 0) {
+      uint64_t t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > limit_ns) {
+        atomicExch(status, unsigned(SHARQ_ERR_TIMEOUT));
+        return;
+      }
+    }
+    __nanosleep(1000);
+  }
+}
+}  // namespace
+}  // namespace sharq
+
 extern "C" {
 
 const char* sharq_status_string(sharq_status s) {
@@ -474,6 +498,18 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   p.tiles_n = N / BN;
   return from_cuda(launch_gemm(maps, p, a->cfg.fmt, a->cfg.mask, res, y_dtype == SHARQ_F32,
                                d.num_sms, st));
+}
+
+sharq_status sharq_wait_probe(const uint32_t* flag, uint32_t expected, uint64_t limit_ns,
+                              void* stream) {
+  if (!flag || (reinterpret_cast<uintptr_t>(flag) & 3u) != 0) return SHARQ_ERR_INVALID_ARG;
+  if (limit_ns < 1000000ull || limit_ns > 10000000000ull) return SHARQ_ERR_INVALID_ARG;
+  DeviceInfo d;
+  sharq_status s = device_info(&d);
+  if (s != SHARQ_OK) return s;
+  wait_probe_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(flag, expected, limit_ns,
+                                                                   d.status);
+  return from_cuda(cudaGetLastError());
 }
 
 sharq_status sharq_device_status(void) {

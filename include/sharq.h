@@ -217,6 +217,15 @@ SHARQ_API sharq_status sharq_linear_workspace_size(int32_t M, int32_t N, int32_t
 SHARQ_API sharq_status sharq_linear_noalloc(const sharq_act* act, const sharq_weight* w, void* Y,
                                             sharq_dtype y_dtype, void* stream);
 
+/* Failure-detection self-test (no counterpart in the pages): launches one thread that
+ * waits until the device word *flag equals `expected`, for at most limit_ns nanoseconds
+ * (1 ms ... 10 s). On expiry it records SHARQ_ERR_TIMEOUT in the device status word and
+ * returns, exactly as the GEMM's bounded pipeline waits do, so that a test can exercise
+ * the detection path (sharq_device_status reports the timeout, the context stays usable)
+ * without a fault. flag: device pointer, 4-byte aligned. Asynchronous on `stream`. */
+SHARQ_API sharq_status sharq_wait_probe(const uint32_t* flag, uint32_t expected,
+                                        uint64_t limit_ns, void* stream);
+
 /* Synchronises the device, returns and clears the status word the kernels write on a
  * bounded-wait timeout (SHARQ_OK or SHARQ_ERR_TIMEOUT), or SHARQ_ERR_CUDA if the
  * synchronisation itself fails. */

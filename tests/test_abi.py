@@ -136,6 +136,14 @@ def test_prepare_rmsnorm_argument_checks(sq):
     assert f(p(0x1000), p(0x8000), 1e-6, sq.BF16, p(0x7000), ctypes.byref(elem), None) == 2
 
 
+def test_wait_probe_argument_checks(sq):
+    p = ctypes.c_void_p
+    assert sq.sharq_wait_probe(None, 1, 10_000_000, None) == 1
+    assert sq.sharq_wait_probe(p(0x1002), 1, 10_000_000, None) == 1  # misaligned
+    assert sq.sharq_wait_probe(p(0x1000), 1, 1000, None) == 1        # limit below 1 ms
+    assert sq.sharq_wait_probe(p(0x1000), 1, 20_000_000_000, None) == 1
+
+
 def test_no_cpu_fallback_without_gpu(sq):
     """On a machine without a usable sm_100 GPU the compute calls return an error code
     (CUDA or ARCH) instead of computing anything on the host."""
