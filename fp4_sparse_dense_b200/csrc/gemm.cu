@@ -384,21 +384,27 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
   const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
   if (i >= total) return;
   const float alpha = __fmul_rn(act_ts[0], w_ts[0]);
+  // the partials of up to 8 splits are loaded together (one L2 round trip per batch, not
+  // one per split) and then added in split order, so the sum is the same fixed sequence
   float acc[8];
-  {
-    const float4 a = *reinterpret_cast<const float4*>(ws + i);
-    const float4 b = *reinterpret_cast<const float4*>(ws + i + 4);
-    acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
-    acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
-  }
-  for (int sidx = 1; sidx < splits; ++sidx) {
-    const float* src = ws + size_t(sidx) * total + i;
-    const float4 a = *reinterpret_cast<const float4*>(src);
-    const float4 b = *reinterpret_cast<const float4*>(src + 4);
-    acc[0] = __fadd_rn(acc[0], a.x); acc[1] = __fadd_rn(acc[1], a.y);
-    acc[2] = __fadd_rn(acc[2], a.z); acc[3] = __fadd_rn(acc[3], a.w);
-    acc[4] = __fadd_rn(acc[4], b.x); acc[5] = __fadd_rn(acc[5], b.y);
-    acc[6] = __fadd_rn(acc[6], b.z); acc[7] = __fadd_rn(acc[7], b.w);
+  for (int base = 0; base < splits; base += 8) {
+    float4 v[8][2];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (base + j < splits) {
+        const float4* src = reinterpret_cast<const float4*>(ws + size_t(base + j) * total + i);
+        v[j][0] = __ldcg(src);
+        v[j][1] = __ldcg(src + 1);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (base + j >= splits) break;
+      const float t[8] = {v[j][0].x, v[j][0].y, v[j][0].z, v[j][0].w,
+                          v[j][1].x, v[j][1].y, v[j][1].z, v[j][1].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = (base + j == 0) ? t[e] : __fadd_rn(acc[e], t[e]);
+    }
   }
   if (OUT_F32) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(Y) + i);
