@@ -180,3 +180,26 @@ def test_split_k_decode(M, K, N):
     check_y(y_split.cpu().numpy().astype(np.float64), y64, False)
     check_y(y_plain.cpu().numpy().astype(np.float64), y64, False)
     check_y(y_bf16.float().cpu().numpy().astype(np.float64), y64, True)
+
+
+def test_split_k_workspace_reused_across_shapes():
+    """One workspace, sized for the largest shape, serves several decode shapes in turn; each
+    call's result is independent of what earlier calls left in it."""
+    import fp4_sparse_dense_b200 as sq
+    import torch
+    K, N = 14336, 4096
+    cfg = cfg_of("nvfp4", "pair48")
+    rng = np.random.default_rng(123)
+    w = gaussian_weight(rng, K, N)
+    wt = sq.quantize_weight(to_device(w), cfg)
+    qw = S.quantize_weight(w.values)
+    ws = sq.linear_workspace(64, N, K, cfg)
+    for M in (64, 1, 16, 64, 8):
+        x = heavy_activations(rng, M, K, per_row=True)
+        act = sq.prepare(to_device(x), cfg)
+        assert sq.linear_workspace(M, N, K, cfg).numel() <= ws.numel()
+        y = sq.linear(act, wt, out_dtype=torch.float32, workspace=ws).cpu().numpy()
+        torch.cuda.synchronize()
+        assert sq.sharq_device_status() == 0
+        y64 = S.linear(S.prepare(x.values), qw)
+        assert rel_fro(y, y64) <= 1e-5, M
