@@ -274,11 +274,13 @@ class Prepared:
     rq: np.ndarray | None  # uint8 codes [M, K]
     rs: np.ndarray | None  # uint8 scale codes [M, K/residual_block]
     r_deq: np.ndarray | None
+    s_r: np.float32 | None = None  # the residual's own tensor scale (variant), else None
 
 
 def prepare(x: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48, residual: bool = True,
             residual_ref: str = "quantized", amax: np.float32 | None = None,
-            given=None) -> Prepared:
+            given=None, residual_scale: str = "shared", amax_r: np.float32 | None = None
+            ) -> Prepared:
     """Online sparse-dense decomposition of one activation tensor X[M x K].
 
     residual_ref="quantized" is the method (r = x - deq(Q(backbone))); "unquantized"
@@ -289,6 +291,10 @@ def prepare(x: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48, residual: bool 
     deq(Q(x)) is a second, dense FP4 term). `amax` overrides the tensor's max |x|, so
     that a sample of rows can be prepared exactly as inside the whole tensor (rows are
     independent once the tensor constants are fixed).
+
+    residual_scale="own" (NVFP4; the variant with two accumulators): the residual gets its
+    own tensor scale s_r = amax|r| / 2688 (k_r = 448 / amax|r|) instead of sharing s_g;
+    `amax_r` overrides amax|r| for a sample of rows.
     """
     x = np.ascontiguousarray(x, dtype=F32)
     M, K = x.shape
@@ -318,10 +324,16 @@ def prepare(x: np.ndarray, fmt: str = NVFP4, mask: str = PAIR48, residual: bool 
         sub = b_deq if residual_ref == "quantized" else np.where(keep, x, F32(0))
         r = np.where(keep, (x - sub).astype(F32), x).astype(F32)
         Br = residual_block(fmt)
-        rc, rsc, rd = quant_blocks(fmt, r.reshape(M, -1, Br), sc)
+        sc_r = sc
+        if residual_scale == "own" and fmt == NVFP4:
+            sc_r = tensor_scales(amax_of(r) if amax_r is None else F32(amax_r))
+        rc, rsc, rd = quant_blocks(fmt, r.reshape(M, -1, Br), sc_r)
         rq = rc.reshape(M, K)
         rs = rsc.reshape(M, K // Br)
         r_deq = rd.reshape(M, K)
+        s_r = sc_r[0] if sc_r is not sc else None
+        return Prepared(fmt, mask, residual, s_g, keep, meta, bq, bs, b_deq, r, rq, rs, r_deq,
+                        s_r)
     return Prepared(fmt, mask, residual, s_g, keep, meta, bq, bs, b_deq, r, rq, rs, r_deq)
 
 
@@ -411,13 +423,20 @@ def linear(p: Prepared, qw: QWeight, rows: np.ndarray | None = None,
     output to a sample (rows are independent, so sampling is exact).
     """
     A = backbone_values(p)
-    if p.residual:
-        A = A + residual_values(p)
     Wv = weight_values(qw)
-    if rows is not None:
-        A = A[rows]
     if cols is not None:
         Wv = Wv[cols]
+    if p.residual and p.s_r is not None:
+        # two accumulators: each path carries its own tensor scale
+        R = residual_values(p)
+        if rows is not None:
+            A, R = A[rows], R[rows]
+        s_gw = float(qw.s_gw) if qw.fmt == NVFP4 else 1.0
+        return s_gw * (float(p.s_g) * (A @ Wv.T) + float(p.s_r) * (R @ Wv.T))
+    if p.residual:
+        A = A + residual_values(p)
+    if rows is not None:
+        A = A[rows]
     return alpha(p, qw) * (A @ Wv.T)
 
 

@@ -87,3 +87,28 @@ def test_ablation_error_ordering_on_outlier_heavy_inputs(fmt):
     assert method <= static
     assert method <= plain
     assert plain2 <= plain
+
+
+def test_own_residual_scale_is_plain_nvfp4_of_the_residual():
+    """The variant with the residual's own tensor scale quantises r exactly as plain NVFP4
+    (no mask, no residual) quantises the tensor r: two independent paths."""
+    x = _x(64, 1024, seed=8)
+    p = S.prepare(x, S.NVFP4, S.PAIR48, residual_scale="own")
+    q = S.prepare(p.r, S.NVFP4, S.NONE, residual=False)
+    assert np.array_equal(p.rq, q.bq) and np.array_equal(p.rs, q.bs)
+    assert p.s_r == q.s_g
+    assert p.s_r < p.s_g  # amax|r| < amax|x| on outlier-heavy rows
+
+
+def test_own_residual_scale_changes_little_on_outlier_heavy_inputs():
+    """Both variants approximate the same product; on these inputs the E4M3 block scales
+    already carry the residual's range, so the two results are close."""
+    from workloads import gaussian_weight
+    x = _x(64, 1024, seed=9)
+    w = gaussian_weight(np.random.default_rng(10), 1024, 256).values
+    qw = S.quantize_weight(w)
+    y_shared = S.linear(S.prepare(x), qw)
+    y_own = S.linear(S.prepare(x, residual_scale="own"), qw)
+    exact = x.astype(np.float64) @ w.astype(np.float64)
+    e = lambda y: np.linalg.norm(y - exact) / np.linalg.norm(exact)
+    assert abs(e(y_own) - e(y_shared)) < 0.1 * e(y_shared)
