@@ -218,6 +218,9 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    if args.workload not in WORKLOADS:
+        raise SystemExit("the reference arm times the single-linear workloads "
+                         f"({', '.join(WORKLOADS)})")
     from oracle import sharq as S
     M, K, N, _ = WORKLOADS[args.workload]
     x, w = make_inputs(args.workload, rank_seed(0))
@@ -407,13 +410,109 @@ def run_gpu(args):
     return 0
 
 
+def run_stack(args):
+    """One Llama-3-8B-shaped layer per step (config 5): q, k, v share one preparation of the
+    attention input, o has its own, gate and up share the MLP input's, down has its own.
+    Weights rotate over 4 layers (436 MB of FP4 payload), so a step streams its weights from
+    HBM as a model's would. Inputs are synthetic (drawn on the device, outlier channels per
+    row); they are not chained from layer to layer (there are no norms between them here)."""
+    import torch
+    import fp4_sparse_dense_b200 as sq
+    from workloads import LLAMA8B_LINEARS
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    M = args.m
+    cfg = sq.Config.from_names(args.fmt, args.mask,
+                               {"on": True, "off": False, "unquantized": "unquantized"}[args.residual])
+    g = torch.Generator(device=dev).manual_seed(5000 + M)
+    shapes = {nm: (k, n) for nm, k, n in LLAMA8B_LINEARS}
+    groups = [("attn", 4096, ["q", "k", "v"]), ("o", 4096, ["o"]), ("mlp", 4096, ["gate", "up"]),
+              ("down", 14336, ["down"])]
+    layers = 4
+
+    def act_input(K):
+        x = torch.randn(M, K, device=dev, generator=g)
+        out = torch.rand(M, K, device=dev, generator=g) < 0.005
+        gain = 20 + 30 * torch.rand(M, K, device=dev, generator=g)
+        return torch.where(out, x * gain, x).to(torch.bfloat16)
+
+    X = {gname: act_input(K) for gname, K, _ in groups}
+    A = {gname: sq.empty_act(M, K, cfg, dev) for gname, K, _ in groups}
+    QW = []
+    for _ in range(layers):
+        lw = {}
+        for nm, (k, n) in shapes.items():
+            w = (torch.randn(k, n, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+            lw[nm] = sq.quantize_weight(w, cfg)
+            del w
+        QW.append(lw)
+    Y = {nm: torch.empty(M, n, dtype=torch.bfloat16, device=dev) for nm, (k, n) in shapes.items()}
+    WS = {nm: sq.linear_workspace(M, n, k, cfg, dev) for nm, (k, n) in shapes.items()}
+    flops = sum(2.0 * M * k * n for k, n in shapes.values())
+    wbytes = 0
+    for t in (QW[0][nm] for nm in shapes):
+        wbytes += sum(b.numel() for b in (t.codes, t.scales_dense, t.scales_sparse) if b is not None)
+
+    def layer(i):
+        lw = QW[i % layers]
+        for gname, _, names in groups:
+            a = sq.prepare(X[gname], cfg, out=A[gname])
+            for nm in names:
+                sq.linear(a, lw[nm], out=Y[nm], workspace=WS[nm])
+
+    for i in range(args.warmup):
+        layer(i)
+    torch.cuda.synchronize()
+    assert sq.sharq_device_status() == 0
+    stream = torch.cuda.current_stream()
+    with Clocks(0) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            layer(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert sq.sharq_device_status() == 0
+    per_layer_ms = ms / args.steps
+    hbm, bf16, bf16_sus, peak_src = load_peaks()
+    value = flops * args.steps / (ms * 1e-3) / 1e12
+    hbm_bound = M < 256  # weight stream dominates below the ridge point (~850 flop/byte)
+    achieved = (wbytes / (per_layer_ms * 1e-3) / 1e9) if hbm_bound else value
+    peak = hbm if hbm_bound else bf16_sus * FP4_OVER_BF16
+    n_prep = sum(len(prep_kernels(args.fmt, args.mask)) for _ in groups)
+    n_gemm = sum(1 + (1 if WS[nm] is not None else 0) for nm in shapes)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_layer_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
+        "data": "synthetic (drawn on the device)",
+        "config": {"workload": "stack8b", "M": M, "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
+                   "layers_rotated": layers, "format": args.fmt, "mask": args.mask,
+                   "residual": args.residual, "out": "bf16",
+                   "l2": f"weights rotate over {layers} layers ({layers * wbytes / 1e6:.0f} MB > 126 MB L2)",
+                   "parallelism": "dp1"},
+        "roofline": {"bound": "hbm" if hbm_bound else "tensor", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s" if hbm_bound else "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None,
+                     "note": ("FP4 weight payload (codes and both scale views) per layer / layer "
+                              "time" if hbm_bound else "2MNK of the 7 linears / layer time"),
+                     "weight_bytes_per_layer": wbytes},
+        "gpu_launches": (n_prep + n_gemm) * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
-    ap.add_argument("--workload", default="mlp_gate_up", choices=list(WORKLOADS))
+    ap.add_argument("--workload", default="mlp_gate_up", choices=list(WORKLOADS) + ["stack8b"])
+    ap.add_argument("--m", type=int, default=1, help="token rows of --workload stack8b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--mask", default="pair48",
@@ -427,6 +526,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "stack8b":
+        return run_stack(args)
     return run_gpu(args)
 
 

@@ -203,3 +203,4 @@ def test_split_k_workspace_reused_across_shapes():
         assert sq.sharq_device_status() == 0
         y64 = S.linear(S.prepare(x.values), qw)
         assert rel_fro(y, y64) <= 1e-5, M
+
