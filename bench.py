@@ -428,6 +428,11 @@ def run_stack(args):
     shapes = {nm: (k, n) for nm, k, n in LLAMA8B_LINEARS}
     groups = [("attn", 4096, ["q", "k", "v"]), ("o", 4096, ["o"]), ("mlp", 4096, ["gate", "up"]),
               ("down", 14336, ["down"])]
+    if args.fused:  # deployment layout: q|k|v and gate|up weights concatenated along N
+        shapes = {"qkv": (4096, 6144), "o": (4096, 4096), "gate_up": (4096, 28672),
+                  "down": (14336, 4096)}
+        groups = [("attn", 4096, ["qkv"]), ("o", 4096, ["o"]), ("mlp", 4096, ["gate_up"]),
+                  ("down", 14336, ["down"])]
     layers = 4
 
     def act_input(K):
@@ -487,7 +492,8 @@ def run_stack(args):
         "warmup": args.warmup, "ms_per_step": per_layer_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
         "data": "synthetic (drawn on the device)",
-        "config": {"workload": "stack8b", "M": M, "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
+        "config": {"workload": "stack8b", "M": M, "fused": bool(args.fused),
+                   "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
                    "layers_rotated": layers, "format": args.fmt, "mask": args.mask,
                    "residual": args.residual, "out": "bf16",
                    "l2": f"weights rotate over {layers} layers ({layers * wbytes / 1e6:.0f} MB > 126 MB L2)",
@@ -513,6 +519,8 @@ def main():
     ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
     ap.add_argument("--workload", default="mlp_gate_up", choices=list(WORKLOADS) + ["stack8b"])
     ap.add_argument("--m", type=int, default=1, help="token rows of --workload stack8b")
+    ap.add_argument("--fused", action="store_true",
+                    help="stack8b: q|k|v and gate|up weights concatenated (4 GEMMs per layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--mask", default="pair48",
