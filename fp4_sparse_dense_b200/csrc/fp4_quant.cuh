@@ -249,17 +249,29 @@ __device__ __forceinline__ void decode8(uint32_t codes, const BlockScale& b, flo
   }
 }
 
-// max |v| over N values (N a multiple of 2) with the three-input max of sm_100.
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float t;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(t) : "f"(a), "f"(b), "f"(c));
+  return t;
+}
+
+// max |v| over N values (N = 16 or 32) with the three-input max of sm_100, as a tree of
+// depth 3-4 (the preparation is latency-bound; a chain would be N/2 deep)
 template <int N>
 __device__ __forceinline__ float amax_n(const float* v) {
-  float a = 0.f;
+  static_assert(N == 16 || N == 32, "block of 16 or 32");
+  constexpr int T = N / 3;  // full triples
+  float m[T + 1];
 #pragma unroll
-  for (int i = 0; i < N; i += 2) {
-    float t;
-    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(t) : "f"(a), "f"(v[i]), "f"(v[i + 1]));
-    a = t;
+  for (int i = 0; i < T; ++i) m[i] = max3_abs(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  m[T] = max3_abs(v[N - 2], v[N - 1], 0.f);  // N % 3 == 1 or 2: rest (overlap is harmless)
+  if (N == 16) {  // 6 partial maxima
+    return fmaxf(max3_abs(m[0], m[1], m[2]), max3_abs(m[3], m[4], m[5]));
   }
-  return a;
+  // N == 32: 11 partial maxima
+  const float n0 = max3_abs(m[0], m[1], m[2]), n1 = max3_abs(m[3], m[4], m[5]);
+  const float n2 = max3_abs(m[6], m[7], m[8]), n3 = max3_abs(m[9], m[10], 0.f);
+  return fmaxf(max3_abs(n0, n1, n2), n3);
 }
 
 // byte offset of (row r, column c) inside a staged tile of 128 rows x C scale columns
