@@ -294,13 +294,14 @@ __device__ __forceinline__ void unpack16(const uint4* c, uint32_t* w) {
 template <bool BF16, bool NORM, bool ABL>
 __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
   const bool mask_given = ABL && p.mask_given;  // ablation flags compile away unless ABL
-  // the quantisation kernel may start its prologue now; it waits for this grid's completion
-  // (griddepcontrol.wait) before it reads anything written here
-  ptx::griddep_launch_dependents();
   __shared__ uint32_t s_top2[64];
   if (threadIdx.x < 64) s_top2[threadIdx.x] = top2_entry(threadIdx.x);
   __syncthreads();
   ptx::griddep_wait();  // X (and rstd) come from the kernels launched before
+  // Only now may the quantisation kernel start: once it runs, the kernels that produced X
+  // have completed, so it may read X before its own wait. It waits (griddepcontrol.wait)
+  // for this grid's completion before it reads anything written here.
+  ptx::griddep_launch_dependents();
   const PairWalk wk(p);
   uint32_t mx = 0;
   int q = wk.q0, row = wk.row0;
@@ -360,19 +361,20 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   __shared__ float s_amax;
   if (threadIdx.x < 64) s_top2[threadIdx.x] = top2_entry(threadIdx.x);
   if (threadIdx.x < 16) s_nib[threadIdx.x] = nibble_entry(threadIdx.x);
-  // NVFP4: launched as a programmatic dependent of prep_mask_kernel; everything above runs
-  // while that kernel finishes, the wait below returns once its writes are visible
+  const PairWalk wk(p);
+  int q = wk.q0, row = wk.row0;
+  uint4 cur[4];
+  // NVFP4: launched as a programmatic dependent of prep_mask_kernel, which releases it only
+  // after its own wait, so X is final here and the first item's load overlaps that kernel's
+  // tail; the wait below returns once the mask kernel's writes (amax, metadata) are visible.
+  // MXFP4 is the first kernel of the call: X may come from the kernel launched just before.
+  if (NV) wk.load(wk.first, row, q, cur);
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();  // the GEMM that follows may start its prologue
-  if (NV && threadIdx.x == 0) {
-    AmaxState* st = reinterpret_cast<AmaxState*>(p.tensor_scale + 2);
-    s_amax = __uint_as_float(*reinterpret_cast<volatile unsigned*>(&st->acc));
-    __threadfence();  // the read above completes before this CTA is counted
-    if (atomicAdd(&st->done, 1u) == gridDim.x - 1) {  // every CTA has read acc
-      st->acc = 0u;
-      st->done = 0u;
-    }
-  }
+  if (!NV) wk.load(wk.first, row, q, cur);
+  AmaxState* const amax_st = reinterpret_cast<AmaxState*>(p.tensor_scale + 2);
+  if (NV && threadIdx.x == 0)
+    s_amax = __uint_as_float(*reinterpret_cast<volatile unsigned*>(&amax_st->acc));
   __syncthreads();
   TensorConsts tc{1.f, 1.f};
   if constexpr (NV) {
@@ -387,7 +389,6 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   }
   __syncthreads();  // decision and scale tables ready
 
-  const PairWalk wk(p);
   const int K = wk.K, M = wk.M, u = wk.u;
   const uint32_t scols_b = uint32_t(K) / 32 / 4;  // 512-byte chunks per 128 rows (backbone)
   const uint32_t scols_r = uint32_t(K) / RB / 4;  // (residual)
@@ -407,9 +408,6 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
     return __ldcg(reinterpret_cast<const unsigned short*>(wk.bm + wk.meta_off(q, r)));
   };
 
-  int q = wk.q0, row = wk.row0;
-  uint4 cur[4];
-  wk.load(wk.first, row, q, cur);
   uint32_t cmeta = load_meta(wk.first, row, q);
 
 #pragma unroll 1
@@ -541,6 +539,15 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
     cmeta = nmeta;
     q = nq;
     row = nrow;
+  }
+  // NVFP4: the last CTA to finish resets the amax state for the next call (every CTA read
+  // acc at its start; the fence orders that read before this CTA is counted)
+  if (NV && threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&amax_st->done, 1u) == gridDim.x - 1) {
+      amax_st->acc = 0u;
+      amax_st->done = 0u;
+    }
   }
 }
 
