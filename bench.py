@@ -31,6 +31,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "SharQ linear TFLOPS (2MNK/t) and % FP4 peak; prep kernel HBM GB/s"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+L2_BYTES = 126 * 2**20  # B200 L2
 
 
 def prep_bytes_per_elem(fmt: str, mask: str, residual: bool) -> float:
@@ -169,6 +170,11 @@ def max_over_ranks(ms: float, dist_mod, device) -> float:
 def job_throughput(flops_per_step: float, world: int, steps: int, ms_max: float) -> float:
     """Whole-job TFLOP/s: all ranks' work divided by the slowest rank's time."""
     return flops_per_step * world * steps / (ms_max * 1e-3) / 1e12
+
+
+def act_tensors(a):
+    """The device buffers of a prepared activation (None where the configuration has none)."""
+    return [t for t in (a.bq, a.bs, a.bm, a.rq, a.rs) if t is not None]
 
 
 def make_inputs(workload: str, seed: int):
@@ -332,6 +338,29 @@ def run_gpu(args):
     torch.cuda.synchronize()
     prep_ms = [e[0].elapsed_time(e[1]) for e in ev]
     gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
+
+    # the preparation alone, calls back to back (as in a layer, where each one's launch hides
+    # behind the previous kernel) over enough input sets that every call reads X from HBM
+    xb = M * K * 2 + sum(t.numel() * t.element_size() for t in act_tensors(ACT[0]))
+    n_prep = max(2, -(-int(2.5 * L2_BYTES) // xb))
+    XP = [X[j % n_sets] if j < n_sets else torch.empty_like(X[0]).copy_(X[j % n_sets])
+          for j in range(n_prep)]
+    AP = [ACT[j] if j < n_sets else sq.empty_act(M, K, cfg, dev) for j in range(n_prep)]
+    if args.mask == "pair48_given":
+        for a in AP[n_sets:]:
+            a.bm.copy_(ACT[0].bm)
+    n_pc = max(3 * n_prep, min(args.steps, 200))
+    for j in range(n_prep):
+        sq.prepare(XP[j], cfg, out=AP[j])
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for j in range(n_pc):
+        sq.prepare(XP[j % n_prep], cfg, out=AP[j % n_prep])
+    p1.record(stream)
+    torch.cuda.synchronize()
+    prep_b2b = p0.elapsed_time(p1) / n_pc
+    del XP, AP
     flops = 2.0 * M * N * K
     value = job_throughput(flops, world, args.steps, ms_max)
 
@@ -360,7 +389,8 @@ def run_gpu(args):
         hbm, bf16, bf16_sus, peak_src = load_peaks()
         fp4_peak = bf16_sus * FP4_OVER_BF16
         gemm_avg = float(np.mean(gemm_ms))
-        prep_avg = float(np.mean(prep_ms))
+        prep_avg = prep_b2b
+        prep_in_step = float(np.mean(prep_ms))
         gemm_tflops = flops / (gemm_avg * 1e-3) / 1e12
         bpe = prep_bytes_per_elem(args.fmt, args.mask, has_res)
         prep_gbs = M * K * bpe / (prep_avg * 1e-3) / 1e9
@@ -384,10 +414,12 @@ def run_gpu(args):
             "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
                      "frac": prep_gbs / hbm,
                      "bytes_per_elem": bpe,
+                     "ms_in_step": prep_in_step,
                      "kernel": " + ".join(prep_kernels(args.fmt, args.mask)),
-                     "note": "two launches (mask, metadata and tensor amax; then quantisation, "
-                             "started early by programmatic dependent launch); algorithmic "
-                             "bytes count X once"},
+                     "note": "ms: calls back to back over input sets larger than L2 (X read "
+                             "from HBM every call); ms_in_step: between events around the "
+                             "call inside the step, which adds the first kernel's launch "
+                             "gap; algorithmic bytes count X once"},
             "gemm_tflops": gemm_tflops,
             "pct_fp4_peak": 100.0 * gemm_tflops / fp4_peak,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
