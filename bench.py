@@ -172,6 +172,34 @@ def job_throughput(flops_per_step: float, world: int, steps: int, ms_max: float)
     return flops_per_step * world * steps / (ms_max * 1e-3) / 1e12
 
 
+def run_pipelined(n, slots, prep, gemm):
+    """n items, the preparation of item j+1 on a side stream (launched to share the SMs,
+    sharq_prepare_alongside) while the GEMMs of item j run on the current stream. prep(j, s)
+    writes activation slot j % slots on stream s; gemm(j) reads it. A slot is rewritten only
+    after the GEMMs that read it are done; the side stream joins the current one at the end."""
+    import torch
+    main = torch.cuda.current_stream()
+    side = run_pipelined.side = getattr(run_pipelined, "side", None) or torch.cuda.Stream()
+    ready = [torch.cuda.Event() for _ in range(slots)]
+    done = [torch.cuda.Event() for _ in range(slots)]
+    side.wait_stream(main)
+    with torch.cuda.stream(side):
+        prep(0, side)
+        ready[0].record(side)
+    for i in range(n):
+        j = i + 1
+        if j < n:
+            with torch.cuda.stream(side):
+                if j >= slots:
+                    side.wait_event(done[j % slots])
+                prep(j, side)
+                ready[j % slots].record(side)
+        main.wait_event(ready[i % slots])
+        gemm(i)
+        done[i % slots].record(main)
+    main.wait_stream(side)
+
+
 def act_tensors(a):
     """The device buffers of a prepared activation (None where the configuration has none)."""
     return [t for t in (a.bq, a.bs, a.bm, a.rq, a.rs) if t is not None]
@@ -312,12 +340,25 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    def timed_steps(k):
+        if args.pipeline:
+            run_pipelined(k, n_sets,
+                          lambda j, s: sq.prepare(X[j % n_sets], cfg, out=ACT[j % n_sets],
+                                                  stream=s, alongside=True),
+                          lambda j: sq.linear(ACT[j % n_sets], QW[j % 2], out=Y[j % n_sets],
+                                              workspace=WS))
+        else:
+            for i in range(k):
+                sq.linear(step(i), QW[i % 2], out=Y[i % n_sets], workspace=WS)
+
+    if args.pipeline:  # warm the two-stream schedule too
+        timed_steps(args.warmup)
+        torch.cuda.synchronize()
     with Clocks(local) as clk:
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         t_start.record(stream)
-        for i in range(args.steps):
-            sq.linear(step(i), QW[i % 2], out=Y[i % n_sets], workspace=WS)
+        timed_steps(args.steps)
         t_end.record(stream)
         torch.cuda.synchronize()
     if world > 1:
@@ -403,6 +444,8 @@ def run_gpu(args):
             "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": args.fmt,
                        "mask": args.mask, "residual": args.residual, "out": "bf16",
                        "l2": f"{n_sets} rotating input sets (> 126 MB L2 per step)",
+                       "schedule": ("pipelined: step i+1's preparation beside step i's GEMM "
+                                    "(two streams)") if args.pipeline else "serial",
                        "parallelism": f"dp{world}"},
             "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
@@ -497,16 +540,32 @@ def run_stack(args):
             for nm in names:
                 sq.linear(a, lw[nm], out=Y[nm], workspace=WS[nm])
 
-    for i in range(args.warmup):
-        layer(i)
+    ng = len(groups)
+
+    def layers_run(k):
+        if args.pipeline:  # group t+1's preparation beside group t's GEMMs, across layers
+            def prep(t, s):
+                gname, _, _ = groups[t % ng]
+                sq.prepare(X[gname], cfg, out=A[gname], stream=s, alongside=True)
+
+            def gemms(t):
+                gname, _, names = groups[t % ng]
+                lw = QW[(t // ng) % layers]
+                for nm in names:
+                    sq.linear(A[gname], lw[nm], out=Y[nm], workspace=WS[nm])
+            run_pipelined(k * ng, ng, prep, gemms)
+        else:
+            for i in range(k):
+                layer(i)
+
+    layers_run(args.warmup)
     torch.cuda.synchronize()
     assert sq.sharq_device_status() == 0
     stream = torch.cuda.current_stream()
     with Clocks(0) as clk:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(args.steps):
-            layer(i)
+        layers_run(args.steps)
         e1.record(stream)
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
@@ -525,6 +584,7 @@ def run_stack(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
         "data": "synthetic (drawn on the device)",
         "config": {"workload": "stack8b", "M": M, "fused": bool(args.fused),
+                   "schedule": "pipelined" if args.pipeline else "serial",
                    "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
                    "layers_rotated": layers, "format": args.fmt, "mask": args.mask,
                    "residual": args.residual, "out": "bf16",
@@ -554,6 +614,9 @@ def main():
     ap.add_argument("--fused", action="store_true",
                     help="stack8b: q|k|v and gate|up weights concatenated (4 GEMMs per layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pipeline", action="store_true",
+                    help="two streams: the next step's (stack8b: group's) preparation runs "
+                         "beside the current GEMM (sharq_prepare_alongside)")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--mask", default="pair48",
                     choices=["pair48", "elem24", "pair48_given", "none"],

@@ -21,12 +21,12 @@ from ._abi import (  # noqa: F401
     sharq_act, sharq_act_bytes, sharq_config, sharq_weight, sharq_weight_bytes, check,
     sharq_act_sizes, sharq_weight_sizes, sharq_status_string, sharq_device_status,
     sharq_prepare, sharq_quantize_weight, sharq_linear, sharq_linear_workspace_size,
-    sharq_linear_noalloc, sharq_prepare_rmsnorm, sharq_wait_probe,
+    sharq_linear_noalloc, sharq_prepare_rmsnorm, sharq_wait_probe, sharq_prepare_alongside,
 )
 
 __all__ = [
     "Config", "QuantWeight", "PreparedAct", "quantize_weight", "prepare", "prepare_rmsnorm",
-    "linear", "sharq_prepare_rmsnorm",
+    "linear", "sharq_prepare_rmsnorm", "sharq_prepare_alongside",
     "sharq_act_sizes", "sharq_weight_sizes", "sharq_prepare", "sharq_quantize_weight",
     "sharq_linear", "sharq_linear_workspace_size", "sharq_linear_noalloc", "sharq_device_status",
     "sharq_status_string", "SharqError", "linear_workspace",
@@ -150,13 +150,17 @@ def quantize_weight(W, cfg: Config = Config(), out: QuantWeight | None = None,
     return out
 
 
-def prepare(X, cfg: Config = Config(), out: PreparedAct | None = None, stream=None) -> PreparedAct:
-    """X: CUDA tensor [M x K] (bf16/fp16) -> backbone / residual FP4 operands."""
+def prepare(X, cfg: Config = Config(), out: PreparedAct | None = None, stream=None,
+            alongside: bool = False) -> PreparedAct:
+    """X: CUDA tensor [M x K] (bf16/fp16) -> backbone / residual FP4 operands.
+    alongside=True: launched to share the GPU with a GEMM running on another stream
+    (sharq_prepare_alongside; identical results)."""
     M, K = X.shape
     X = X.contiguous()
     out = out or empty_act(M, K, cfg, X.device)
     ca = out.c()
-    check(sharq_prepare(_ptr(X), _dtype_code(X), ctypes.byref(ca), _stream(stream)))
+    fn = sharq_prepare_alongside if alongside else sharq_prepare
+    check(fn(_ptr(X), _dtype_code(X), ctypes.byref(ca), _stream(stream)))
     return out
 
 

@@ -710,11 +710,11 @@ __global__ void __launch_bounds__(256) prep_elem_kernel(PrepParams p) {
 // launch with the programmatic-stream-serialization attribute: the kernel may start while
 // the previous one in the stream finishes and waits (griddepcontrol.wait) for its results
 template <typename... Args>
-static cudaError_t launch_pdl(void (*kern)(Args...), unsigned blocks, cudaStream_t st,
-                              Args... args) {
+static cudaError_t launch_pdl_t(void (*kern)(Args...), unsigned blocks, unsigned threads,
+                                cudaStream_t st, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(threads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -723,23 +723,39 @@ static cudaError_t launch_pdl(void (*kern)(Args...), unsigned blocks, cudaStream
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
+template <typename... Args>
+static cudaError_t launch_pdl(void (*kern)(Args...), unsigned blocks, cudaStream_t st,
+                              Args... args) {
+  return launch_pdl_t(kern, blocks, 256u, st, args...);
+}
 
 // CTAs of a persistent preparation kernel: enough warp items for every warp, at most what
-// fits on the GPU at once (resident CTAs per SM from the occupancy calculator, cached)
+// fits on the GPU at once (resident CTAs per SM from the occupancy calculator, cached).
+// Beside a GEMM (p.alongside): one CTA per SM of `threads` threads. The kernels prefer the
+// largest shared-memory carveout, so that an SM running one of them can still take a GEMM
+// CTA that needs nearly all of its shared memory without reconfiguring.
 template <typename Kern>
 static cudaError_t persistent_blocks(Kern kern, int* per_sm, const PrepParams& p, int num_sms,
-                                     unsigned* blocks) {
+                                     unsigned* blocks, unsigned threads = 256) {
   if (*per_sm == 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, 256, 0);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         int(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, 256, 0);
     if (e != cudaSuccess) return e;
     if (*per_sm < 1) *per_sm = 1;
   }
   const long items = long(p.Mp / 4) * (p.K / 256);
-  long b = (items + 7) / 8;
-  const long cap = long(num_sms) * *per_sm;
+  const long warps = threads / 32;
+  long b = (items + warps - 1) / warps;
+  const long cap = long(num_sms) * (p.alongside ? 1 : *per_sm);
   *blocks = unsigned(b < cap ? b : cap);
   return cudaSuccess;
 }
+
+// threads per CTA of the quantisation kernel: beside a GEMM the SM has about 16 K registers
+// left, so 128 threads (4 warps at up to 80 registers); alone 256
+static unsigned quant_threads(const PrepParams& p) { return p.alongside ? 128u : 256u; }
 
 template <bool BF16, int FMT, bool RES, bool NORM, bool ABL>
 static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
@@ -761,8 +777,9 @@ static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cud
     auto kern = prep_pair_kernel<BF16, FMT, RES, NORM, ABL>;
     static int per_sm = 0;
     unsigned blocks = 0;
-    if ((e = persistent_blocks(kern, &per_sm, p, num_sms, &blocks)) != cudaSuccess) return e;
-    e = launch_pdl(kern, blocks, st, p);
+    const unsigned qt = quant_threads(p);
+    if ((e = persistent_blocks(kern, &per_sm, p, num_sms, &blocks, qt)) != cudaSuccess) return e;
+    e = launch_pdl_t(kern, blocks, qt, st, p);
     if (e != cudaSuccess) return e;
   } else {
     if (NORM) return cudaErrorNotSupported;

@@ -221,10 +221,11 @@ using namespace sharq;
 
 namespace sharq {
 namespace {
-// Both preparation entry points: gamma == nullptr prepares X as given; otherwise the
-// RMSNorm of X with (gamma, eps), writing the per-row rstd.
+// The preparation entry points: gamma == nullptr prepares X as given; otherwise the
+// RMSNorm of X with (gamma, eps), writing the per-row rstd. alongside: launch sized to
+// share the SMs with a GEMM running on another stream (same results).
 sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, const void* gamma,
-                          float eps, float* rstd, void* stream) {
+                          float eps, float* rstd, void* stream, bool alongside = false) {
   if (!X || !a) return SHARQ_ERR_INVALID_ARG;
   if (dtype != SHARQ_F16 && dtype != SHARQ_BF16) return SHARQ_ERR_INVALID_ARG;
   sharq_act_bytes sz;
@@ -278,6 +279,7 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
   p.mask_given = a->cfg.mask == SHARQ_MASK_PAIR_4_8_GIVEN;
   p.keep_all = none;
   p.res_unquant = a->cfg.residual == 2;
+  p.alongside = alongside ? 1 : 0;
   return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
 }
 }  // namespace
@@ -367,6 +369,11 @@ sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, const sharq
 
 sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* a, void* stream) {
   return sharq::prepare_impl(X, dtype, a, nullptr, 0.f, nullptr, stream);
+}
+
+sharq_status sharq_prepare_alongside(const void* X, sharq_dtype dtype, const sharq_act* a,
+                                    void* stream) {
+  return sharq::prepare_impl(X, dtype, a, nullptr, 0.f, nullptr, stream, true);
 }
 
 sharq_status sharq_prepare_rmsnorm(const void* X, const void* gamma, float eps, sharq_dtype dtype,

@@ -29,6 +29,7 @@ struct PrepParams {
   int mask_given;       // pair mask read from bm instead of chosen per row
   int keep_all;         // no mask: every element on the (dense) backbone
   int res_unquant;      // residual against the unquantised backbone
+  int alongside;        // launch sized to run beside a GEMM on another stream
 };
 
 struct WeightQuantParams {

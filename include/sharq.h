@@ -163,6 +163,18 @@ SHARQ_API sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, c
  * mask M * K must be below 2^31 (else SHARQ_ERR_UNSUPPORTED). */
 SHARQ_API sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* act, void* stream);
 
+/* The same preparation, with results identical to sharq_prepare, launched to share the GPU
+ * with a sharq_linear GEMM that runs at the same time on another stream (the overlap of
+ * one batch's preparation with another batch's GEMM: the SharQ page's Fig. 4a latency
+ * breakdown puts the preparation beside the two GEMMs). The persistent pair-mask kernels
+ * run one CTA per SM, small enough in registers and shared memory to sit beside a GEMM
+ * CTA, so neither waits for the other to leave the SMs. Alone on the GPU it is slower than
+ * sharq_prepare. Arguments, buffers and errors as for sharq_prepare; the caller orders the
+ * two streams (the GEMM that reads *act waits for this call, and a call that rewrites *act
+ * waits for the GEMMs reading it). The element 2:4 mask runs its usual kernel. */
+SHARQ_API sharq_status sharq_prepare_alongside(const void* X, sharq_dtype dtype, const sharq_act* act,
+                                   void* stream);
+
 /* Preparation with the layer's RMSNorm absorbed (SharQ page, abstract: the fused
  * preparation operator takes in layer normalisation; RMSNorm is that of the Llama/Qwen
  * models the page evaluates). The prepared input is y = round16((x * rstd) * gamma) per
