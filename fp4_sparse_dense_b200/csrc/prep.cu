@@ -709,39 +709,40 @@ __global__ void __launch_bounds__(256) prep_elem_kernel(PrepParams p) {
 
 // launch with the programmatic-stream-serialization attribute: the kernel may start while
 // the previous one in the stream finishes and waits (griddepcontrol.wait) for its results
+// Beside a GEMM (alongside) the launch also asks for the largest shared-memory carveout, so
+// that an SM running one of these CTAs can still take a GEMM CTA that needs nearly all of
+// its shared memory without reconfiguring; alone the default split keeps L1 large for the
+// X stream.
 template <typename... Args>
 static cudaError_t launch_pdl_t(void (*kern)(Args...), unsigned blocks, unsigned threads,
-                                cudaStream_t st, Args... args) {
+                                bool alongside, cudaStream_t st, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
   cfg.blockDim = dim3(threads);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributePreferredSharedMemoryCarveout;
+  attr[1].val.sharedMemCarveout = unsigned(cudaSharedmemCarveoutMaxShared);
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = alongside ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 template <typename... Args>
 static cudaError_t launch_pdl(void (*kern)(Args...), unsigned blocks, cudaStream_t st,
                               Args... args) {
-  return launch_pdl_t(kern, blocks, 256u, st, args...);
+  return launch_pdl_t(kern, blocks, 256u, false, st, args...);
 }
 
 // CTAs of a persistent preparation kernel: enough warp items for every warp, at most what
 // fits on the GPU at once (resident CTAs per SM from the occupancy calculator, cached).
-// Beside a GEMM (p.alongside): one CTA per SM of `threads` threads. The kernels prefer the
-// largest shared-memory carveout, so that an SM running one of them can still take a GEMM
-// CTA that needs nearly all of its shared memory without reconfiguring.
+// Beside a GEMM (p.alongside): one CTA per SM of `threads` threads.
 template <typename Kern>
 static cudaError_t persistent_blocks(Kern kern, int* per_sm, const PrepParams& p, int num_sms,
                                      unsigned* blocks, unsigned threads = 256) {
   if (*per_sm == 0) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                         int(cudaSharedmemCarveoutMaxShared));
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, 256, 0);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, 256, 0);
     if (e != cudaSuccess) return e;
     if (*per_sm < 1) *per_sm = 1;
   }
@@ -772,14 +773,14 @@ static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cud
       static int mk_per_sm = 0;
       unsigned mb = 0;
       if ((e = persistent_blocks(mk, &mk_per_sm, p, num_sms, &mb)) != cudaSuccess) return e;
-      if ((e = launch_pdl(mk, mb, st, p)) != cudaSuccess) return e;
+      if ((e = launch_pdl_t(mk, mb, 256u, p.alongside != 0, st, p)) != cudaSuccess) return e;
     }
     auto kern = prep_pair_kernel<BF16, FMT, RES, NORM, ABL>;
     static int per_sm = 0;
     unsigned blocks = 0;
     const unsigned qt = quant_threads(p);
     if ((e = persistent_blocks(kern, &per_sm, p, num_sms, &blocks, qt)) != cudaSuccess) return e;
-    e = launch_pdl_t(kern, blocks, qt, st, p);
+    e = launch_pdl_t(kern, blocks, qt, p.alongside != 0, st, p);
     if (e != cudaSuccess) return e;
   } else {
     if (NORM) return cudaErrorNotSupported;
