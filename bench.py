@@ -53,9 +53,11 @@ def metric_ceiling(mask: str, residual: bool) -> float:
     return 1.0 / t
 
 
-def prep_kernels(fmt: str, mask: str) -> list:
+def prep_kernels(fmt: str, mask: str, residual: str = "on") -> list:
     if mask.startswith("pair48"):
-        return (["prep_mask_kernel"] if fmt == "nvfp4" else []) + ["prep_pair_kernel"]
+        # the residual's own tensor scale runs the quantisation twice (amax|r| in between)
+        quant = ["prep_pair_kernel"] * (2 if residual == "own" else 1)
+        return (["prep_mask_kernel"] if fmt == "nvfp4" else []) + quant
     return (["amax_kernel"] if fmt == "nvfp4" else []) + ["prep_elem_kernel"]
 
 
@@ -87,9 +89,11 @@ GEMM_SRC = ["fp4_sparse_dense_b200/csrc/gemm.cu", "fp4_sparse_dense_b200/csrc/ge
             "fp4_sparse_dense_b200/csrc/sharq_internal.h"]
 
 
-def gemm_kernel_name(M: int, N: int) -> str:
-    """Which GEMM kernel sharq_linear launches for this shape (CTA pair for M >= 256)."""
-    return "sharq_gemm_pair_kernel" if M >= 256 and N % 256 == 0 else "sharq_gemm_kernel"
+def gemm_kernel_name(M: int, N: int, residual: str = "on") -> str:
+    """Which GEMM kernel sharq_linear launches for this shape (CTA pair for M >= 256; the
+    two-accumulator variant of the residual's own scale always runs the one-CTA kernel)."""
+    pair = M >= 256 and N % 256 == 0 and residual != "own"
+    return "sharq_gemm_pair_kernel" if pair else "sharq_gemm_kernel"
 
 
 def traffic_from_profile(workload: str):
@@ -219,6 +223,8 @@ def oracle_modes(args) -> dict:
     kw = {"fmt": args.fmt, "mask": args.mask, "residual": args.residual != "off"}
     if args.residual == "unquantized":
         kw["residual_ref"] = "unquantized"
+    if args.residual == "own":  # amax|r| over each sampled block of rows
+        kw["residual_scale"] = "own"
     return kw
 
 
@@ -298,7 +304,7 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     dev = torch.device("cuda", local)
     M, K, N, _ = WORKLOADS[args.workload]
-    res_mode = {"on": True, "off": False, "unquantized": "unquantized"}[args.residual]
+    res_mode = {"on": True, "off": False, "unquantized": "unquantized", "own": "own"}[args.residual]
     cfg = sq.Config.from_names(args.fmt, args.mask, res_mode)  # default: the method
     has_res = args.residual != "off"
 
@@ -435,7 +441,9 @@ def run_gpu(args):
         gemm_tflops = flops / (gemm_avg * 1e-3) / 1e12
         bpe = prep_bytes_per_elem(args.fmt, args.mask, has_res)
         prep_gbs = M * K * bpe / (prep_avg * 1e-3) / 1e9
-        traffic = traffic_from_profile(args.workload)
+        # the committed capture is of the method's kernel (NVFP4, pair 4:8, residual on)
+        method = (args.fmt, args.mask, args.residual) == ("nvfp4", "pair48", "on")
+        traffic = traffic_from_profile(args.workload) if method else None
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
@@ -453,12 +461,12 @@ def run_gpu(args):
                          "peak_source": f"{peak_src}: bf16 sustained {bf16_sus} x "
                                         f"{FP4_OVER_BF16} (nominal FP4:BF16)",
                          "ceiling_frac": metric_ceiling(args.mask, has_res),
-                         "kernel": gemm_kernel_name(M, N), "kernel_ms": gemm_avg},
+                         "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg},
             "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
                      "frac": prep_gbs / hbm,
                      "bytes_per_elem": bpe,
                      "ms_in_step": prep_in_step,
-                     "kernel": " + ".join(prep_kernels(args.fmt, args.mask)),
+                     "kernel": " + ".join(prep_kernels(args.fmt, args.mask, args.residual)),
                      "note": "ms: calls back to back over input sets larger than L2 (X read "
                              "from HBM every call); ms_in_step: between events around the "
                              "call inside the step, which adds the first kernel's launch "
@@ -467,7 +475,7 @@ def run_gpu(args):
             "pct_fp4_peak": 100.0 * gemm_tflops / fp4_peak,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
                     "d2h_bytes_per_step": M * N * 2},
-            "gpu_launches": (len(prep_kernels(args.fmt, args.mask)) + 1 +
+            "gpu_launches": (len(prep_kernels(args.fmt, args.mask, args.residual)) + 1 +
                              (1 if WS is not None else 0)) * args.steps,
             "clocks": clk.summary(),
         }
@@ -498,7 +506,8 @@ def run_stack(args):
     dev = torch.device("cuda", 0)
     M = args.m
     cfg = sq.Config.from_names(args.fmt, args.mask,
-                               {"on": True, "off": False, "unquantized": "unquantized"}[args.residual])
+                               {"on": True, "off": False, "unquantized": "unquantized",
+                                "own": "own"}[args.residual])
     g = torch.Generator(device=dev).manual_seed(5000 + M)
     shapes = {nm: (k, n) for nm, k, n in LLAMA8B_LINEARS}
     groups = [("attn", 4096, ["q", "k", "v"]), ("o", 4096, ["o"]), ("mlp", 4096, ["gate", "up"]),
@@ -576,7 +585,7 @@ def run_stack(args):
     hbm_bound = M < 256  # weight stream dominates below the ridge point (~850 flop/byte)
     achieved = (wbytes / (per_layer_ms * 1e-3) / 1e9) if hbm_bound else value
     peak = hbm if hbm_bound else bf16_sus * FP4_OVER_BF16
-    n_prep = sum(len(prep_kernels(args.fmt, args.mask)) for _ in groups)
+    n_prep = sum(len(prep_kernels(args.fmt, args.mask, args.residual)) for _ in groups)
     n_gemm = sum(1 + (1 if WS[nm] is not None else 0) for nm in shapes)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
@@ -622,7 +631,8 @@ def main():
                     choices=["pair48", "elem24", "pair48_given", "none"],
                     help="pair48 is the method; the others are ablations / baselines "
                          "(none with --residual off: plain FP4)")
-    ap.add_argument("--residual", default="on", choices=["on", "off", "unquantized"])
+    ap.add_argument("--residual", default="on", choices=["on", "off", "unquantized", "own"],
+                    help="own: the residual with its own tensor scale (two accumulators)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:

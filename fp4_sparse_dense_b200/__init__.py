@@ -36,8 +36,9 @@ __all__ = [
 
 @dataclass(frozen=True)
 class Config:
-    """fmt, mask and residual mode of sharq_config. residual: True (the method), False, or
-    "unquantized" (ablation: residual against the unquantised backbone). Masks
+    """fmt, mask and residual mode of sharq_config. residual: True (the method), False,
+    "unquantized" (ablation: residual against the unquantised backbone) or "own" (the
+    residual with its own tensor scale, two accumulators; NVFP4 with a pair mask). Masks
     "pair48_given" and "none" are ablations (see include/sharq.h)."""
     fmt: int = NVFP4
     mask: int = PAIR_4_8
@@ -46,6 +47,8 @@ class Config:
     def c(self) -> sharq_config:
         if self.residual == "unquantized":
             r = 2
+        elif self.residual == "own":
+            r = 3
         else:
             r = 1 if self.residual else 0
         return sharq_config(self.fmt, self.mask, r)

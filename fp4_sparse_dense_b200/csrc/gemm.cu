@@ -21,6 +21,9 @@
 // Tensor memory: columns [0, BN) accumulator; from column 256 two buffers of the scale
 // factors and sparse metadata, used by alternate K steps, so that the copies of step k+1
 // never write columns the MMAs of step k may still read.
+// TWO (the variant whose residual has its own tensor scale s_r, BN = 128): the residual's
+// MMAs accumulate in columns [128, 256) and the epilogue forms
+// s_gw * (s_g * acc_backbone + s_r * acc_residual).
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -83,13 +86,14 @@ struct GemmCfg {
   static constexpr uint32_t SCALE_FMT = NV ? 0u : (1u << 23);  // E4M3 or E8M0 scales
 };
 
-template <int FMT, bool PAIR, bool RES, int BN, bool OUT_F32>
+template <int FMT, bool PAIR, bool RES, int BN, bool OUT_F32, bool TWO = false>
 __global__ void __launch_bounds__(kThreads, 1)
     sharq_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_r,
                       const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   using C = GemmCfg<FMT, PAIR, RES, BN>;
+  static_assert(!TWO || (RES && BN == 128), "second accumulator: residual on, BN = 128");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -275,18 +279,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (RES) {
+            // one accumulator, or (TWO) the residual's own, starting at the range's first step
+            const uint32_t tacc = TWO ? tbase + uint32_t(BN) : tbase;
+            uint32_t acc_r = TWO ? (kt > kt0 ? 1u : 0u) : 1u;
             for (int i = 0; i < 4; ++i) {
               const uint64_t a = ptx::smem_desc(st + C::OFF_R + 32 * i, 16, 1024, 2);
               const uint64_t b = ptx::smem_desc(st + C::OFF_W + 32 * i, 16, 1024, 2);
               if (C::NV) {
-                ptx::mma_nvf4(tbase, a, b, idesc_d, tb + C::COL_SFR + 4 * i,
-                              tb + C::COL_SWD + i * (BN / 32), 1u);
+                ptx::mma_nvf4(tacc, a, b, idesc_d, tb + C::COL_SFR + 4 * i,
+                              tb + C::COL_SWD + i * (BN / 32), acc_r);
               } else {
                 const uint32_t id = 2u * uint32_t(i & 1);
-                ptx::mma_mxf4(tbase, a, b, idesc_d | (id << 29) | (id << 4),
+                ptx::mma_mxf4(tacc, a, b, idesc_d | (id << 29) | (id << 4),
                               (tb + C::COL_SFR + 4 * (i >> 1)) | (id << 30),
-                              (tb + C::COL_SWD + (i >> 1) * (BN / 32)) | (id << 30), 1u);
+                              (tb + C::COL_SWD + (i >> 1) * (BN / 32)) | (id << 30), acc_r);
               }
+              acc_r = 1u;
             }
           }
           ptx::mma_commit(ptx::smem_u32(empty_bar + s));
@@ -326,16 +334,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t v[HALF];
 #pragma unroll
       for (int c = 0; c < HALF / 32; ++c) ptx::tmem_ld_32x32b_x32(taddr + c * 32, v + 32 * c);
+      if constexpr (TWO) {
+        uint32_t vr[HALF];
+#pragma unroll
+        for (int c = 0; c < HALF / 32; ++c)
+          ptx::tmem_ld_32x32b_x32(taddr + uint32_t(BN) + c * 32, vr + 32 * c);
+        ptx::tmem_ld_wait();
+        // s_gw * (s_g * b + s_r * r), then stored with a unit scale
+        const float ab = alpha, ar = __fmul_rn(p.act_ts[6], p.w_ts[0]);
+#pragma unroll
+        for (int i = 0; i < HALF; ++i)
+          v[i] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(v[i]), ab),
+                                           __fmul_rn(__uint_as_float(vr[i]), ar)));
+      }
       ptx::tmem_ld_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_u32(tempty_bar));
+      const float out_scale = TWO ? 1.0f : alpha;
       if (p.splits > 1)  // unscaled FP32 partial of this K range, reduced by a second kernel
         store_rows_f32<HALF>(p.ws + size_t(ks) * p.M * p.N, p.M, p.N, v, 1.0f, row,
                              nb * BN + half * HALF);
       else if (OUT_F32)
-        store_rows_f32<HALF>(static_cast<float*>(p.Y), p.M, p.N, v, alpha, row, nb * BN + half * HALF);
+        store_rows_f32<HALF>(static_cast<float*>(p.Y), p.M, p.N, v, out_scale, row, nb * BN + half * HALF);
       else
-        store_rows_bf16<HALF>(&tm_y, epi_stage, v, alpha, mb * 128 + quarter * 32, nb * BN + half * HALF, lane);
+        store_rows_bf16<HALF>(&tm_y, epi_stage, v, out_scale, mb * 128 + quarter * 32, nb * BN + half * HALF, lane);
     }
     if (!OUT_F32 && p.splits == 1 && lane == 0) ptx::bulk_wait_all();  // stores done before exit
     if (!ok && lane == 0) atomicExch(p.status, unsigned(SHARQ_ERR_TIMEOUT));
@@ -349,10 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int FMT, bool PAIR, bool RES, int BN, bool OUT_F32>
+template <int FMT, bool PAIR, bool RES, int BN, bool OUT_F32, bool TWO = false>
 static cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, int num_sms, cudaStream_t st) {
   using C = GemmCfg<FMT, PAIR, RES, BN>;
-  auto kern = sharq_gemm_kernel<FMT, PAIR, RES, BN, OUT_F32>;
+  auto kern = sharq_gemm_kernel<FMT, PAIR, RES, BN, OUT_F32, TWO>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n * p.splits;
@@ -448,6 +470,15 @@ static cudaError_t launch_m(const GemmMaps& m, const GemmParams& p, int mask, bo
                             int n, cudaStream_t st) {
   return is_pair_mask(mask) ? launch_r<FMT, true>(m, p, res, f32, n, st)
                                      : launch_r<FMT, false>(m, p, res, f32, n, st);
+}
+
+// The variant whose residual has its own tensor scale: NVFP4, pair mask, BN = 128, two
+// accumulators, no split-K.
+cudaError_t launch_gemm_two(const GemmMaps& maps, const GemmParams& p, bool out_f32, int num_sms,
+                            cudaStream_t st) {
+  if (p.splits != 1 || p.tiles_n * 128 != p.N) return cudaErrorInvalidValue;
+  return out_f32 ? launch_t<SHARQ_NVFP4, true, true, 128, true, true>(maps, p, num_sms, st)
+                 : launch_t<SHARQ_NVFP4, true, true, 128, false, true>(maps, p, num_sms, st);
 }
 
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int mask,

@@ -14,6 +14,7 @@
 // segment); codes are written with 8/16-byte stores, coalesced along the row; scales and
 // metadata are staged in shared memory and written as contiguous 16-byte vectors.
 #include <cstdint>
+#include <type_traits>
 #include <cuda_runtime.h>
 
 #include "fp4_device.cuh"
@@ -354,11 +355,18 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   constexpr bool NV = FMT == SHARQ_NVFP4;
   // ablation flags compile away unless ABL (the method's instantiation stays lean)
   const bool mask_given = ABL && p.mask_given, res_unquant = ABL && p.res_unquant;
+  // residual with its own tensor scale (NVFP4, the two-accumulator variant): phase 1 writes
+  // the backbone and folds max |r| into a second amax state; phase 2 recomputes the same
+  // backbone and r and writes the residual quantised with s_r = amax|r| / 2688
+  const int res_phase = (ABL && NV && RESIDUAL) ? p.res_phase : 0;
   constexpr int RB = NV ? 16 : 32;  // residual block
   __shared__ uint32_t s_top2[64];
   __shared__ uint32_t s_nib[16];
   __shared__ NvScaleTable s_nv;
-  __shared__ float s_amax;
+  struct NoTable {};
+  __shared__ std::conditional_t<ABL && NV && RESIDUAL, NvScaleTable, NoTable> s_nvr;
+  __shared__ float s_amax, s_amax_r;
+  __shared__ unsigned s_rmax[8];
   if (threadIdx.x < 64) s_top2[threadIdx.x] = top2_entry(threadIdx.x);
   if (threadIdx.x < 16) s_nib[threadIdx.x] = nibble_entry(threadIdx.x);
   const PairWalk wk(p);
@@ -373,14 +381,28 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   ptx::griddep_launch_dependents();  // the GEMM that follows may start its prologue
   if (!NV) wk.load(wk.first, row, q, cur);
   AmaxState* const amax_st = reinterpret_cast<AmaxState*>(p.tensor_scale + 2);
-  if (NV && threadIdx.x == 0)
-    s_amax = __uint_as_float(*reinterpret_cast<volatile unsigned*>(&amax_st->acc));
+  AmaxState* const amax_r_st = reinterpret_cast<AmaxState*>(p.tensor_scale + 4);
+  if (NV && threadIdx.x == 0) {
+    if (res_phase == 2) {  // amax|X| as phase 1 wrote it; amax|r| from phase 1's reduction
+      s_amax = *reinterpret_cast<volatile float*>(p.tensor_scale + 1);
+      s_amax_r = __uint_as_float(*reinterpret_cast<volatile unsigned*>(&amax_r_st->acc));
+    } else {
+      s_amax = __uint_as_float(*reinterpret_cast<volatile unsigned*>(&amax_st->acc));
+    }
+  }
   __syncthreads();
-  TensorConsts tc{1.f, 1.f};
+  TensorConsts tc{1.f, 1.f}, tcr{1.f, 1.f};
   if constexpr (NV) {
     tc = tensor_consts(s_amax);
     nv_table_fill(&s_nv, tc.s_g, threadIdx.x);
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (res_phase == 2) {
+      tcr = tensor_consts(s_amax_r);
+      if constexpr (ABL && RESIDUAL) nv_table_fill(&s_nvr, tcr.s_g, threadIdx.x);
+      if (blockIdx.x == 0 && threadIdx.x == 0) {
+        p.tensor_scale[6] = tcr.s_g;
+        p.tensor_scale[7] = s_amax_r;
+      }
+    } else if (blockIdx.x == 0 && threadIdx.x == 0) {
       p.tensor_scale[0] = tc.s_g;
       p.tensor_scale[1] = s_amax;
     }
@@ -388,6 +410,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
     p.tensor_scale[0] = 1.0f;
   }
   __syncthreads();  // decision and scale tables ready
+  float r_max = 0.f;  // phase 1: running max |r| of this thread
 
   const int K = wk.K, M = wk.M, u = wk.u;
   const uint32_t scols_b = uint32_t(K) / 32 / 4;  // 512-byte chunks per 128 rows (backbone)
@@ -397,6 +420,13 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
   auto scale_of = [&](float a) {
     if constexpr (NV) return nv_block_scale(a, tc, &s_nv);
     else return block_scale<FMT>(a, tc);
+  };
+  // the residual's blocks: the backbone's table, or phase 2's table of s_r
+  auto scale_of_r = [&](float a) {
+    if constexpr (NV && ABL && RESIDUAL) {
+      if (res_phase == 2) return nv_block_scale(a, tcr, &s_nvr);
+    }
+    return scale_of(a);
   };
   auto decode_of = [&](uint32_t codes, const BlockScale& b, float* out) {
     if constexpr (NV) decode8_nv(codes, b, tc.s_g, out);
@@ -462,9 +492,10 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
       // selector takes bytes i0, i1 of the first word and 4 + i0, 4 + i1 of the second)
       const uint32_t sel01 = __byte_perm(L[0], L[1], 0x0062u) + 0x4400u;
       const uint32_t sel23 = __byte_perm(L[2], L[3], 0x0062u) + 0x4400u;
-      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.bq) +
-                                (uint32_t(row) * uint32_t(K / 4) + k0 / 4)) =
-          make_uint2(__byte_perm(c[0], c[1], sel01), __byte_perm(c[2], c[3], sel23));
+      if (res_phase != 2)
+        *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.bq) +
+                                  (uint32_t(row) * uint32_t(K / 4) + k0 / 4)) =
+            make_uint2(__byte_perm(c[0], c[1], sel01), __byte_perm(c[2], c[3], sel23));
       if (RESIDUAL) {
         // ---- residual against the quantised backbone
         float r[32];
@@ -487,22 +518,27 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
           }
         }
         uint32_t rc[4];
+        if (res_phase == 1) {
+          r_max = fmaxf(r_max, amax_n<32>(r));
+        } else {
 #pragma unroll
-        for (int hb = 0; hb < 32 / RB; ++hb) {
-          const BlockScale rb = scale_of(amax_n<RB>(r + hb * RB));
-          if (hb == 0) rsf0 = rb.code; else rsf1 = rb.code;
+          for (int hb = 0; hb < 32 / RB; ++hb) {
+            const BlockScale rb = scale_of_r(amax_n<RB>(r + hb * RB));
+            if (hb == 0) rsf0 = rb.code; else rsf1 = rb.code;
 #pragma unroll
-          for (int g = 0; g < RB / 8; ++g) rc[hb * (RB / 8) + g] = encode8(r + hb * RB + 8 * g, rb);
+            for (int g = 0; g < RB / 8; ++g)
+              rc[hb * (RB / 8) + g] = encode8(r + hb * RB + 8 * g, rb);
+          }
+          *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.rq) +
+                                    (uint32_t(row) * uint32_t(K / 2) + k0 / 2)) =
+              make_uint4(rc[0], rc[1], rc[2], rc[3]);
         }
-        *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.rq) +
-                                  (uint32_t(row) * uint32_t(K / 2) + k0 / 2)) =
-            make_uint4(rc[0], rc[1], rc[2], rc[3]);
       }
     }
 
     // ---- scales (and MXFP4 metadata): gather neighbouring lanes' bytes into 32-bit stores
     const uint32_t rq32 = uint32_t(row & 31) * 16u + uint32_t((row >> 5) & 3) * 4u;
-    {
+    if (res_phase != 2) {
       // backbone scale column q*8+u: lanes u..u+3 form one 4-byte word
       uint32_t word = bsf;
       word |= __shfl_down_sync(0xFFFFFFFFu, bsf, 1) << 8;
@@ -513,7 +549,7 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
         *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(p.bs) + (chunk * 512u + rq32)) = word;
       }
     }
-    if (RESIDUAL) {
+    if (RESIDUAL && res_phase != 1) {
       if constexpr (RB == 16) {
         // residual scale columns q*16+2u, +1: lanes u, u+1 form one 4-byte word
         const uint32_t two = rsf0 | (rsf1 << 8);
@@ -540,13 +576,25 @@ __global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
     q = nq;
     row = nrow;
   }
-  // NVFP4: the last CTA to finish resets the amax state for the next call (every CTA read
-  // acc at its start; the fence orders that read before this CTA is counted)
+  if (res_phase == 1) {  // fold max |r| into the second amax state (one atomic per CTA)
+    uint32_t h = __float_as_uint(r_max);
+    for (int off = 16; off; off >>= 1) h = max(h, __shfl_xor_sync(0xFFFFFFFFu, h, off));
+    if ((threadIdx.x & 31) == 0) s_rmax[threadIdx.x >> 5] = h;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t b = 0;
+      for (int i = 0; i < int(blockDim.x >> 5); ++i) b = max(b, s_rmax[i]);
+      atomicMax(&amax_r_st->acc, b);
+    }
+  }
+  // NVFP4: the last CTA to finish resets the amax state it read for the next call (every
+  // CTA read acc at its start; the fence orders that read before this CTA is counted)
   if (NV && threadIdx.x == 0) {
+    AmaxState* const st = res_phase == 2 ? amax_r_st : amax_st;
     __threadfence();
-    if (atomicAdd(&amax_st->done, 1u) == gridDim.x - 1) {
-      amax_st->acc = 0u;
-      amax_st->done = 0u;
+    if (atomicAdd(&st->done, 1u) == gridDim.x - 1) {
+      st->acc = 0u;
+      st->done = 0u;
     }
   }
 }
@@ -762,13 +810,13 @@ template <bool BF16, int FMT, bool RES, bool NORM, bool ABL>
 static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
   if (is_pair_mask(mask)) {
     cudaError_t e = cudaSuccess;
-    if (NORM) {  // per-row rstd first: one warp per row
+    if (NORM && p.res_phase != 2) {  // per-row rstd first: one warp per row
       long rb = (long(p.M) + 7) / 8;
       if (rb > long(num_sms) * 8) rb = long(num_sms) * 8;
       e = launch_pdl(rms_kernel<BF16>, unsigned(rb), st, p);
       if (e != cudaSuccess) return e;
     }
-    if (FMT == SHARQ_NVFP4) {
+    if (FMT == SHARQ_NVFP4 && p.res_phase != 2) {
       auto mk = prep_mask_kernel<BF16, NORM, ABL>;
       static int mk_per_sm = 0;
       unsigned mb = 0;
@@ -792,7 +840,7 @@ static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cud
 
 template <bool BF16, int FMT, bool RES, bool NORM>
 static cudaError_t launch_prep_a(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
-  const bool abl = p.mask_given || p.res_unquant;
+  const bool abl = p.mask_given || p.res_unquant || p.res_phase != 0;
   return abl ? launch_prep_t<BF16, FMT, RES, NORM, true>(p, mask, num_sms, st)
              : launch_prep_t<BF16, FMT, RES, NORM, false>(p, mask, num_sms, st);
 }

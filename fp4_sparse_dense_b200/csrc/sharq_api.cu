@@ -61,7 +61,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 sharq_status check_cfg(sharq_config c) {
   if (c.fmt != SHARQ_NVFP4 && c.fmt != SHARQ_MXFP4) return SHARQ_ERR_INVALID_ARG;
   if (c.mask < SHARQ_MASK_PAIR_4_8 || c.mask > SHARQ_MASK_NONE) return SHARQ_ERR_INVALID_ARG;
-  if (c.residual < 0 || c.residual > 2) return SHARQ_ERR_INVALID_ARG;
+  if (c.residual < 0 || c.residual > 3) return SHARQ_ERR_INVALID_ARG;
+  // the residual's own tensor scale exists for NVFP4 (MXFP4 has no tensor scale) and is
+  // built for the pair mask
+  if (c.residual == 3 && (c.fmt != SHARQ_NVFP4 || !is_pair_mask(c.mask)))
+    return SHARQ_ERR_UNSUPPORTED;
   return SHARQ_OK;
 }
 
@@ -280,6 +284,16 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
   p.keep_all = none;
   p.res_unquant = a->cfg.residual == 2;
   p.alongside = alongside ? 1 : 0;
+  p.res_phase = 0;
+  if (a->cfg.residual != 3)
+    return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
+  // the residual's own tensor scale: amax|r| is a grid-wide reduction that follows the
+  // backbone's quantisation, so the quantisation runs twice (backbone + amax|r|, then the
+  // residual with s_r)
+  p.res_phase = 1;
+  if ((s = from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st))) != SHARQ_OK)
+    return s;
+  p.res_phase = 2;
   return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
 }
 }  // namespace
@@ -392,7 +406,7 @@ sharq_status sharq_linear_workspace_size(int32_t M, int32_t N, int32_t K, sharq_
   if ((s = weight_sizes(K, N, cfg, &wsz)) != SHARQ_OK) return s;
   DeviceInfo d;
   if ((s = device_info(&d)) != SHARQ_OK) return s;
-  const int splits = plan_splits(M, N, K, d.num_sms);
+  const int splits = cfg.residual == 3 ? 1 : plan_splits(M, N, K, d.num_sms);
   *bytes = splits > 1 ? size_t(splits) * size_t(M) * size_t(N) * sizeof(float) : 0;
   return SHARQ_OK;
 }
@@ -439,7 +453,8 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   p.ws = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  if (M >= 256 && N % 256 == 0) {
+  const bool own = a->cfg.residual == 3;  // residual with its own tensor scale
+  if (M >= 256 && N % 256 == 0 && !own) {
     // CTA-pair kernel: 256 x 256 tiles, half of the weight tile per CTA
     const bool nv = a->cfg.fmt == SHARQ_NVFP4;
     const uint32_t dch_rows = uint32_t(256 / (nv ? 16 : 32) / 4) * 2;  // 256-byte rows per K step
@@ -477,7 +492,8 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
                                       d.num_sms, st));
   }
 
-  const int BN = (N % 256 == 0) ? 256 : 128;
+  // two accumulators (own residual scale) take 128 + 128 tensor-memory columns: BN = 128
+  const int BN = (N % 256 == 0 && !own) ? 256 : 128;
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   if ((s = make_map(&maps.w, w->codes, uint64_t(K) / 2, uint64_t(N), 128, uint32_t(BN),
@@ -496,13 +512,14 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   {
     const int splits = plan_splits(M, N, K, d.num_sms);
     const size_t need = size_t(splits) * size_t(M) * size_t(N) * sizeof(float);
-    if (splits > 1 && workspace && workspace_bytes >= need && aligned16(workspace)) {
+    if (splits > 1 && !own && workspace && workspace_bytes >= need && aligned16(workspace)) {
       p.splits = splits;
       p.ws = static_cast<float*>(workspace);
     }
   }
   p.tiles_m = (M + 127) / 128;
   p.tiles_n = N / BN;
+  if (own) return from_cuda(launch_gemm_two(maps, p, y_dtype == SHARQ_F32, d.num_sms, st));
   return from_cuda(launch_gemm(maps, p, a->cfg.fmt, a->cfg.mask, res, y_dtype == SHARQ_F32,
                                d.num_sms, st));
 }

@@ -30,6 +30,7 @@ struct PrepParams {
   int keep_all;         // no mask: every element on the (dense) backbone
   int res_unquant;      // residual against the unquantised backbone
   int alongside;        // launch sized to run beside a GEMM on another stream
+  int res_phase;        // residual with its own tensor scale: 1 backbone + amax|r|, 2 residual
 };
 
 struct WeightQuantParams {
@@ -69,6 +70,9 @@ cudaError_t launch_weight_quant(const WeightQuantParams& p, bool bf16, int fmt, 
 struct GemmMaps {
   CUtensorMap w, b, r, y;  // y: bf16 output, 32 x 32 boxes (unused for float output)
 };
+// residual with its own tensor scale (two accumulators), NVFP4 pair mask, 128-wide tiles
+cudaError_t launch_gemm_two(const GemmMaps& maps, const GemmParams& p, bool out_f32, int num_sms,
+                            cudaStream_t st);
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int mask,
                         bool residual, bool out_f32, int num_sms, cudaStream_t st);
 

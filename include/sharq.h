@@ -81,7 +81,11 @@ typedef struct {
   int32_t mask;     /* sharq_mask */
   int32_t residual; /* 1: backbone + residual (the method); 0: backbone only;
                        2: ablation, residual against the unquantised backbone
-                       (r = x - backbone: 0 where the mask keeps, x elsewhere) */
+                       (r = x - backbone: 0 where the mask keeps, x elsewhere);
+                       3: the residual with its own tensor scale s_r = amax|r| / 2688
+                       instead of sharing s_g (NVFP4 with a pair mask, else
+                       SHARQ_ERR_UNSUPPORTED): two accumulators, Y = s_gw * (s_g *
+                       acc_backbone + s_r * acc_residual) */
 } sharq_config;
 
 /* Block sizes along K (logical positions per scale), fixed by the MMA consuming them:
@@ -128,9 +132,11 @@ typedef struct {
   void* rs;            /* residual scales, tiled, M x K/residual_block */
   float* tensor_scale; /* 8 floats (32 bytes): [0] s_g = amax|X| / 2688 (NVFP4) or 1.0
                           (MXFP4); [1] amax|X| (NVFP4); both written by sharq_prepare.
-                          [2..7] library state of the amax reduction: set them to zero once
-                          when the buffer is allocated and never write them afterwards
-                          (re-zero them if a call was interrupted by a device error). */
+                          [6] s_r = amax|r| / 2688 and [7] amax|r|, written when
+                          residual == 3. [2..5] library state of the amax reductions: set
+                          [2..7] to zero once when the buffer is allocated and never write
+                          [2..5] afterwards (re-zero them if a call was interrupted by a
+                          device error). */
   int32_t M, K;
   sharq_config cfg;
 } sharq_act;
@@ -192,7 +198,8 @@ SHARQ_API sharq_status sharq_prepare_rmsnorm(const void* X, const void* gamma, f
 /* Y[M x N] = alpha * (sparse-FP4-GEMM(backbone, W) + dense-FP4-GEMM(residual, W)) with
  * alpha = s_g * s_gw, accumulated in FP32 tensor memory and written once (SharQ page, "Core
  * claim": a sparse FP4 GEMM for the backbone and a dense FP4 GEMM for the compensation,
- * sharing one weight payload). Y: device pointer, row-major, y_dtype BF16 (the product) or
+ * sharing one weight payload). With residual == 3 the two GEMMs accumulate separately and
+ * Y = s_gw * (s_g * acc_backbone + s_r * acc_residual) (128-wide tiles, no split-K). Y: device pointer, row-major, y_dtype BF16 (the product) or
  * F32. act->cfg must equal w->cfg and act->K == w->K.
  * workspace / workspace_bytes: optional caller-owned device scratch (16-byte aligned) for
  * the split-K path used when the output has too few tiles to occupy the GPU (decode-sized

@@ -87,14 +87,31 @@ def test_weight_sizes_match_oracle_layouts(sq, fmt, mask):
     assert sz.scales_sparse == (want["scales_sparse"].size if S.is_pair(mask) else 0)
 
 
+@pytest.mark.parametrize("mask", ["pair48", "pair48_given"])
+def test_own_residual_scale_sizes_match_oracle_layouts(sq, mask):
+    """residual == 3 writes the buffers of residual on (its scale goes to tensor_scale[6])."""
+    M, K = 130, 512
+    x = np.random.default_rng(2).standard_normal((M, K)).astype(np.float32)
+    given = S.keep_pairs48(x) if mask == "pair48_given" else None
+    want = S.act_buffers(S.prepare(x, "nvfp4", mask, given=given, residual_scale="own"))
+    sz = sq.sharq_act_bytes()
+    assert sq.sharq_act_sizes(M, K, sq.Config.from_names("nvfp4", mask, "own").c(),
+                              ctypes.byref(sz)) == 0
+    assert (sz.bq, sz.bs, sz.bm, sz.rq, sz.rs) == tuple(
+        want[k].size for k in ("bq", "bs", "bm", "rq", "rs"))
+
+
 def test_bad_shapes_and_configs_rejected(sq):
     sz = sq.sharq_act_bytes()
     ok = sq.Config().c()
     assert sq.sharq_act_sizes(16, 200, ok, ctypes.byref(sz)) == 1   # K % 256
     assert sq.sharq_act_sizes(0, 256, ok, ctypes.byref(sz)) == 1    # M < 1
     assert sq.sharq_act_sizes(16, 256, sq.sharq_config(7, 0, 1), ctypes.byref(sz)) == 1
-    assert sq.sharq_act_sizes(16, 256, sq.sharq_config(0, 0, 3), ctypes.byref(sz)) == 1
+    assert sq.sharq_act_sizes(16, 256, sq.sharq_config(0, 0, 4), ctypes.byref(sz)) == 1
     assert sq.sharq_act_sizes(16, 256, sq.sharq_config(0, 4, 1), ctypes.byref(sz)) == 1
+    # the residual's own tensor scale: NVFP4 with a pair mask only
+    for fmt, mask, code in ((0, 0, 0), (0, 2, 0), (1, 0, 2), (0, 1, 2), (0, 3, 2)):
+        assert sq.sharq_act_sizes(16, 256, sq.sharq_config(fmt, mask, 3), ctypes.byref(sz)) == code
     wz = sq.sharq_weight_bytes()
     assert sq.sharq_weight_sizes(256, 100, ok, ctypes.byref(wz)) == 1  # N % 128
 
