@@ -109,6 +109,23 @@ def traffic_from_profile(workload: str):
     return e.get("dram_bytes_per_launch")
 
 
+PREP_SRC = ["fp4_sparse_dense_b200/csrc/prep.cu", "fp4_sparse_dense_b200/csrc/fp4_quant.cuh",
+            "fp4_sparse_dense_b200/csrc/fp4_device.cuh", "fp4_sparse_dense_b200/csrc/sm100_ptx.cuh",
+            "fp4_sparse_dense_b200/csrc/sharq_internal.h"]
+
+
+def prep_issue_from_profile(workload: str):
+    """Warp instructions per X element of the preparation (all its kernels) from the
+    committed ncu count, when it was taken on the current preparation source (else None)."""
+    p = os.path.join(ROOT, "profiles", "prep_issue.json")
+    if not os.path.exists(p):
+        return None
+    e = json.load(open(p)).get(workload)
+    if not e or e.get("prep_src") != src_hash(PREP_SRC):
+        return None
+    return e.get("warp_instructions_per_elem")
+
+
 class Clocks:
     """nvidia-smi sampling during the timed region."""
 
@@ -444,6 +461,19 @@ def run_gpu(args):
         # the committed capture is of the method's kernel (NVFP4, pair 4:8, residual on)
         method = (args.fmt, args.mask, args.residual) == ("nvfp4", "pair48", "on")
         traffic = traffic_from_profile(args.workload) if method else None
+        clocks = clk.summary()
+        # the preparation is bound by instruction issue, not HBM: its issue-rate roofline
+        # (warp instructions per element from the committed count; peak = 4 issues per SM
+        # per cycle at the median SM clock of the timed region)
+        ipe = prep_issue_from_profile(args.workload) if method else None
+        issue = None
+        if ipe and clocks.get("sm_mhz"):
+            n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+            peak_i = n_sm * 4 * clocks["sm_mhz"] * 1e6
+            ach_i = ipe * M * K / (prep_avg * 1e-3)
+            issue = {"warp_instructions_per_elem": ipe, "achieved_ginst_s": ach_i / 1e9,
+                     "peak_ginst_s": peak_i / 1e9, "frac": ach_i / peak_i,
+                     "peak_source": f"{n_sm} SMs x 4 issue slots x {clocks['sm_mhz']} MHz"}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
@@ -466,6 +496,7 @@ def run_gpu(args):
                      "frac": prep_gbs / hbm,
                      "bytes_per_elem": bpe,
                      "ms_in_step": prep_in_step,
+                     "issue_roofline": issue,
                      "kernel": " + ".join(prep_kernels(args.fmt, args.mask, args.residual)),
                      "note": "ms: calls back to back over input sets larger than L2 (X read "
                              "from HBM every call); ms_in_step: between events around the "
@@ -477,7 +508,7 @@ def run_gpu(args):
                     "d2h_bytes_per_step": M * N * 2},
             "gpu_launches": (len(prep_kernels(args.fmt, args.mask, args.residual)) + 1 +
                              (1 if WS is not None else 0)) * args.steps,
-            "clocks": clk.summary(),
+            "clocks": clocks,
         }
         if not args.no_cpu_baseline and world == 1:
             from oracle import sharq as S
