@@ -601,11 +601,28 @@ def run_stack(args):
     layers_run(args.warmup)
     torch.cuda.synchronize()
     assert sq.sharq_device_status() == 0
+    graph = None
+    if args.graph:
+        # one CUDA graph of `layers` layers (every weight set once): replaying it launches
+        # the same kernels with the same programmatic dependencies, without the host calls
+        if args.steps % layers:
+            args.steps += layers - args.steps % layers
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layers_run(layers)
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+        assert sq.sharq_device_status() == 0
     stream = torch.cuda.current_stream()
     with Clocks(0) as clk:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        layers_run(args.steps)
+        if graph is not None:
+            for _ in range(args.steps // layers):
+                graph.replay()
+        else:
+            layers_run(args.steps)
         e1.record(stream)
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
@@ -625,6 +642,7 @@ def run_stack(args):
         "data": "synthetic (drawn on the device)",
         "config": {"workload": "stack8b", "M": M, "fused": bool(args.fused),
                    "schedule": "pipelined" if args.pipeline else "serial",
+                   "launch": f"CUDA graph of {layers} layers" if args.graph else "eager",
                    "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
                    "layers_rotated": layers, "format": args.fmt, "mask": args.mask,
                    "residual": args.residual, "out": "bf16",
@@ -657,6 +675,9 @@ def main():
     ap.add_argument("--pipeline", action="store_true",
                     help="two streams: the next step's (stack8b: group's) preparation runs "
                          "beside the current GEMM (sharq_prepare_alongside)")
+    ap.add_argument("--graph", action="store_true",
+                    help="stack8b: replay the layers from one CUDA graph (no host calls in the "
+                         "timed region)")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--mask", default="pair48",
                     choices=["pair48", "elem24", "pair48_given", "none"],
