@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
 // (the backbone operand) or in place with zeros elsewhere, which dequantise to the backbone
 // at kept positions and +0 elsewhere, so r = x - deq needs no per-element selection.
 template <bool BF16, int FMT, bool RESIDUAL, bool NORM, bool ABL>
-__global__ void __launch_bounds__(256) prep_pair_kernel(PrepParams p) {
+__global__ void __launch_bounds__(256, ABL ? 1 : 3) prep_pair_kernel(PrepParams p) {
   constexpr bool NV = FMT == SHARQ_NVFP4;
   // ablation flags compile away unless ABL (the method's instantiation stays lean)
   const bool mask_given = ABL && p.mask_given, res_unquant = ABL && p.res_unquant;
