@@ -491,6 +491,11 @@ def run_gpu(args):
                          "peak_source": f"{peak_src}: bf16 sustained {bf16_sus} x "
                                         f"{FP4_OVER_BF16} (nominal FP4:BF16)",
                          "ceiling_frac": metric_ceiling(args.mask, has_res),
+                         # the tensor pipe's executed work (sparse backbone at twice the
+                         # dense rate): 2MNK / ceiling per launch, against the same peak
+                         "executed_frac": gemm_tflops / fp4_peak / metric_ceiling(args.mask, has_res),
+                         # against 4x the measured bf16 burst figure instead of the sustained
+                         "frac_vs_burst_peak": gemm_tflops / (bf16 * FP4_OVER_BF16),
                          "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg},
             "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
                      "frac": prep_gbs / hbm,
