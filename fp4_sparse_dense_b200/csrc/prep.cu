@@ -440,7 +440,9 @@ __global__ void __launch_bounds__(256, ABL ? 1 : 3) prep_pair_kernel(PrepParams 
 
   uint32_t cmeta = load_meta(wk.first, row, q);
 
-#pragma unroll 1
+  // two items per loop trip for the NVFP4 method (measured about 2 % faster on a
+  // 4096 x 4096 tensor), one otherwise
+#pragma unroll (NV && !ABL ? 2 : 1)
   for (int item = wk.first; item < wk.n_items; item += wk.stride) {
     int nq = q, nrow = row;
     wk.advance(nq, nrow);
