@@ -59,7 +59,50 @@ __global__ void __launch_bounds__(512) amax_kernel(const uint4* __restrict__ X, 
   }
 }
 
+// NVFP4 tensor amax across the two preparation kernels, in words 2..3 of the caller's
+// tensor-scale buffer (zero before the first call): the first kernel (the mask kernel, or
+// with RMSNorm absorbed the rstd kernel) folds max |x| into `acc` with atomicMax; every CTA of the quantisation kernel reads it once and counts
+// itself in `done`, and the CTA that completes the count sets both back to zero for the
+// next call. No CTA waits for another.
+struct AmaxState {
+  unsigned acc;   // max |x| as float bits (non-negative floats order like their bits)
+  unsigned done;  // CTAs of the quantisation kernel that have read acc
+};
+
+// CTA max of the threads' packed 15-bit magnitudes (two per word), folded into st->acc.
+template <bool BF16>
+__device__ void block_max_to(uint32_t m, AmaxState* st) {
+  __shared__ unsigned s_red[8];
+  uint32_t h = max(m & 0xFFFFu, m >> 16);
+  for (int off = 16; off; off >>= 1) h = max(h, __shfl_xor_sync(0xFFFFFFFFu, h, off));
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = h;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0;
+    for (int i = 0; i < int(blockDim.x >> 5); ++i) b = max(b, s_red[i]);
+    atomicMax(&st->acc, __float_as_uint(in_to_float<BF16>(b)));
+  }
+}
+
 // ------------------------------------------------------------------------------ RMSNorm
+
+// One word of two 16-bit inputs x normalised with rstd r and weights g:
+// y = round16((x * r) * g) per value (float32 products, one rounding each, then RNE to the
+// input's 16-bit format).
+template <bool BF16>
+__device__ __forceinline__ uint32_t norm_word(uint32_t x, uint32_t g, float r) {
+  const float lo = __fmul_rn(__fmul_rn(in_to_float<BF16>(x & 0xFFFFu), r),
+                             in_to_float<BF16>(g & 0xFFFFu));
+  const float hi = __fmul_rn(__fmul_rn(in_to_float<BF16>(x >> 16), r),
+                             in_to_float<BF16>(g >> 16));
+  uint32_t y;
+  if (BF16) {
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(y) : "f"(hi), "f"(lo));
+  } else {
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(y) : "f"(hi), "f"(lo));
+  }
+  return y;
+}
 
 // Per-row rstd = 1 / sqrt(mean_k x^2 + eps), the RMSNorm that the preparation absorbs (the
 // SharQ page's fused operator takes in layer normalisation; RMSNorm is that of the
@@ -67,14 +110,18 @@ __global__ void __launch_bounds__(512) amax_kernel(const uint4* __restrict__ X, 
 // result is reproducible: chunk c of 8 elements belongs to lane c mod 32, each lane adds
 // its chunks' squares in increasing k, then a butterfly over lanes (xor 16, 8, 4, 2, 1).
 // Squares of 16-bit inputs are exact; every addition and the division, square root and
-// reciprocal round to nearest once.
-template <bool BF16>
+// reciprocal round to nearest once. AMAX (NVFP4): a second pass over the row (from L1/L2)
+// forms the normalised values y exactly as the quantisation kernel will and folds max |y|
+// into the tensor amax, so that no separate mask kernel has to read X again; the
+// quantisation kernel then computes the mask itself.
+template <bool BF16, bool AMAX>
 __global__ void __launch_bounds__(256) rms_kernel(PrepParams p) {
   ptx::griddep_wait();  // X may come from the kernel launched just before
   ptx::griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
   const uint32_t chunks = uint32_t(p.K) / 8;
+  uint32_t mx = 0;  // AMAX: packed 15-bit magnitudes of y
   for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < p.M; row += warps) {
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.X) +
                                                       uint32_t(row) * uint32_t(p.K));
@@ -92,11 +139,22 @@ __global__ void __launch_bounds__(256) rms_kernel(PrepParams p) {
     }
 #pragma unroll
     for (int off = 16; off; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xFFFFFFFFu, acc, off));
-    if (lane == 0) {
-      const float ms = __fdiv_rn(acc, float(p.K));
-      p.rstd[row] = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, p.eps)));
+    // the butterfly leaves the same sum in every lane (each step adds the same two values)
+    const float r = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(acc, float(p.K)), p.eps)));
+    if (lane == 0) p.rstd[row] = r;
+    if (AMAX) {
+      const uint4* g4 = static_cast<const uint4*>(p.gamma);
+#pragma unroll 4
+      for (uint32_t c = lane; c < chunks; c += 32) {
+        const uint4 v = __ldg(src + c), gv = __ldg(g4 + c);
+        mx = __vmaxu2(mx, norm_word<BF16>(v.x, gv.x, r) & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, norm_word<BF16>(v.y, gv.y, r) & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, norm_word<BF16>(v.z, gv.z, r) & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, norm_word<BF16>(v.w, gv.w, r) & 0x7FFF7FFFu);
+      }
     }
   }
+  if (AMAX) block_max_to<BF16>(mx, reinterpret_cast<AmaxState*>(p.tensor_scale + 2));
 }
 
 // y = round16((x * rstd) * gamma) for the 32 inputs of one unit (16 words of two 16-bit
@@ -111,18 +169,7 @@ __device__ __forceinline__ void rms_apply(uint32_t* w, const PrepParams& p, int 
     const uint4 gv = __ldg(g4 + c);
     const uint32_t g[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t& x = w[4 * c + i];
-      const float lo = __fmul_rn(__fmul_rn(in_to_float<BF16>(x & 0xFFFFu), r),
-                                 in_to_float<BF16>(g[i] & 0xFFFFu));
-      const float hi = __fmul_rn(__fmul_rn(in_to_float<BF16>(x >> 16), r),
-                                 in_to_float<BF16>(g[i] >> 16));
-      if (BF16) {
-        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(x) : "f"(hi), "f"(lo));
-      } else {
-        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(x) : "f"(hi), "f"(lo));
-      }
-    }
+    for (int i = 0; i < 4; ++i) w[4 * c + i] = norm_word<BF16>(w[4 * c + i], g[i], r);
   }
 }
 
@@ -163,30 +210,6 @@ __device__ __forceinline__ float hi16(uint32_t w) {
   return BF16 ? __uint_as_float(w & 0xFFFF0000u) : in_to_float<false>(w >> 16);
 }
 
-// NVFP4 tensor amax across the two preparation kernels, in words 2..3 of the caller's
-// tensor-scale buffer (zero before the first call): the mask kernel folds max |x| into
-// `acc` with atomicMax; every CTA of the quantisation kernel reads it once and counts
-// itself in `done`, and the CTA that completes the count sets both back to zero for the
-// next call. No CTA waits for another.
-struct AmaxState {
-  unsigned acc;   // max |x| as float bits (non-negative floats order like their bits)
-  unsigned done;  // CTAs of the quantisation kernel that have read acc
-};
-
-// CTA max of the threads' packed 15-bit magnitudes (two per word), folded into st->acc.
-template <bool BF16>
-__device__ void block_max_to(uint32_t m, AmaxState* st) {
-  __shared__ unsigned s_red[8];
-  uint32_t h = max(m & 0xFFFFu, m >> 16);
-  for (int off = 16; off; off >>= 1) h = max(h, __shfl_xor_sync(0xFFFFFFFFu, h, off));
-  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = h;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t b = 0;
-    for (int i = 0; i < int(blockDim.x >> 5); ++i) b = max(b, s_red[i]);
-    atomicMax(&st->acc, __float_as_uint(in_to_float<BF16>(b)));
-  }
-}
 
 // Table entry of a metadata nibble i0 | i1 << 2 (same packing as top2_entry); nibbles that
 // the mask never produces map to pairs (0, 1).
@@ -432,7 +455,9 @@ __global__ void __launch_bounds__(256, ABL ? 1 : 3) prep_pair_kernel(PrepParams 
     if constexpr (NV) decode8_nv(codes, b, tc.s_g, out);
     else decode8<FMT>(codes, b, tc.s_g, out);
   };
-  const bool meta_in = NV || mask_given;  // mask read back from bm
+  // mask read back from bm (written by prep_mask_kernel, or supplied), else computed here
+  // (MXFP4, and NVFP4 with RMSNorm absorbed, where the rstd kernel supplies the amax)
+  const bool meta_in = (NV && !(NORM && !ABL)) || mask_given;
   auto load_meta = [&](int it, int r, int q) -> uint32_t {
     if (!meta_in || it >= wk.n_items || r >= M) return 0x4444u;
     return __ldcg(reinterpret_cast<const unsigned short*>(wk.bm + wk.meta_off(q, r)));
@@ -812,13 +837,16 @@ template <bool BF16, int FMT, bool RES, bool NORM, bool ABL>
 static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
   if (is_pair_mask(mask)) {
     cudaError_t e = cudaSuccess;
+    // NVFP4 + RMSNorm (the method): the rstd kernel also reduces the tensor amax of the
+    // normalised X, and the quantisation kernel computes the mask (no mask kernel)
+    constexpr bool NORM_AMAX = NORM && !ABL && FMT == SHARQ_NVFP4;
     if (NORM && p.res_phase != 2) {  // per-row rstd first: one warp per row
       long rb = (long(p.M) + 7) / 8;
       if (rb > long(num_sms) * 8) rb = long(num_sms) * 8;
-      e = launch_pdl(rms_kernel<BF16>, unsigned(rb), st, p);
+      e = launch_pdl(rms_kernel<BF16, NORM_AMAX>, unsigned(rb), st, p);
       if (e != cudaSuccess) return e;
     }
-    if (FMT == SHARQ_NVFP4 && p.res_phase != 2) {
+    if (FMT == SHARQ_NVFP4 && !NORM_AMAX && p.res_phase != 2) {
       auto mk = prep_mask_kernel<BF16, NORM, ABL>;
       static int mk_per_sm = 0;
       unsigned mb = 0;
