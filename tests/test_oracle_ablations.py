@@ -112,3 +112,19 @@ def test_own_residual_scale_changes_little_on_outlier_heavy_inputs():
     exact = x.astype(np.float64) @ w.astype(np.float64)
     e = lambda y: np.linalg.norm(y - exact) / np.linalg.norm(exact)
     assert abs(e(y_own) - e(y_shared)) < 0.1 * e(y_shared)
+
+
+def test_two_accumulator_product_is_sparse_part_plus_plain_nvfp4_of_the_residual():
+    """The own-scale variant's Y: its backbone part is the sparse-only product, and its
+    residual part is the product of plain NVFP4 of r (no mask, own tensor scale) with the
+    weight's dense view; both computed by other code paths (the sparse-only product and
+    the no-mask preparation), so a wrong scale or a dropped term fails here."""
+    from workloads import gaussian_weight
+    x = _x(48, 512, seed=11)
+    w = gaussian_weight(np.random.default_rng(12), 512, 128).values
+    p = S.prepare(x, S.NVFP4, S.PAIR48, residual_scale="own")
+    qw = S.quantize_weight(w, S.NVFP4, S.PAIR48)  # one code payload for both paths
+    y = S.linear(p, qw)
+    sparse = S.linear_sparse_only(p, qw)
+    plain_r = S.linear(S.prepare(p.r, S.NVFP4, S.NONE, residual=False), qw)
+    np.testing.assert_allclose(y, sparse + plain_r, rtol=1e-12, atol=1e-12 * np.abs(y).max())
