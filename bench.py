@@ -53,7 +53,9 @@ def metric_ceiling(mask: str, residual: bool) -> float:
     return 1.0 / t
 
 
-def prep_kernels(fmt: str, mask: str, residual: str = "on") -> list:
+def prep_kernels(fmt: str, mask: str, residual: str = "on", given_amax: bool = False) -> list:
+    if given_amax:  # the caller's NVFP4 amax: one kernel with the mask inline
+        return ["prep_pair_kernel"]
     if mask.startswith("pair48"):
         # the residual's own tensor scale runs the quantisation twice (amax|r| in between)
         quant = ["prep_pair_kernel"] * (2 if residual == "own" else 1)
@@ -348,8 +350,12 @@ def run_gpu(args):
     WS = sq.linear_workspace(M, N, K, cfg, dev)  # split-K scratch (None for prefill shapes)
     stream = torch.cuda.current_stream()
 
+    # --given-amax: the NVFP4 tensor amax of each input set reduced beforehand (outside the
+    # timed region, by torch) and passed in; the preparation is then a single kernel
+    AMX = [x.abs().max().float().reshape(1) for x in X] if args.given_amax else [None] * n_sets
+
     def step(i):
-        a = sq.prepare(X[i % n_sets], cfg, out=ACT[i % n_sets])
+        a = sq.prepare(X[i % n_sets], cfg, out=ACT[i % n_sets], amax=AMX[i % n_sets])
         return a
 
     for i in range(args.warmup):
@@ -409,18 +415,19 @@ def run_gpu(args):
     n_prep = max(2, -(-int(2.5 * L2_BYTES) // xb))
     XP = [X[j % n_sets] if j < n_sets else torch.empty_like(X[0]).copy_(X[j % n_sets])
           for j in range(n_prep)]
+    AMP = [AMX[j % n_sets] for j in range(n_prep)]
     AP = [ACT[j] if j < n_sets else sq.empty_act(M, K, cfg, dev) for j in range(n_prep)]
     if args.mask == "pair48_given":
         for a in AP[n_sets:]:
             a.bm.copy_(ACT[0].bm)
     n_pc = max(3 * n_prep, min(args.steps, 200))
     for j in range(n_prep):
-        sq.prepare(XP[j], cfg, out=AP[j])
+        sq.prepare(XP[j], cfg, out=AP[j], amax=AMP[j])
     torch.cuda.synchronize()
     p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     p0.record(stream)
     for j in range(n_pc):
-        sq.prepare(XP[j % n_prep], cfg, out=AP[j % n_prep])
+        sq.prepare(XP[j % n_prep], cfg, out=AP[j % n_prep], amax=AMP[j % n_prep])
     p1.record(stream)
     torch.cuda.synchronize()
     prep_b2b = p0.elapsed_time(p1) / n_pc
@@ -459,7 +466,8 @@ def run_gpu(args):
         bpe = prep_bytes_per_elem(args.fmt, args.mask, has_res)
         prep_gbs = M * K * bpe / (prep_avg * 1e-3) / 1e9
         # the committed capture is of the method's kernel (NVFP4, pair 4:8, residual on)
-        method = (args.fmt, args.mask, args.residual) == ("nvfp4", "pair48", "on")
+        method = ((args.fmt, args.mask, args.residual) == ("nvfp4", "pair48", "on")
+                  and not args.given_amax)
         traffic = traffic_from_profile(args.workload) if method else None
         clocks = clk.summary()
         # the preparation is bound by instruction issue, not HBM: its issue-rate roofline
@@ -484,6 +492,8 @@ def run_gpu(args):
                        "l2": f"{n_sets} rotating input sets (> 126 MB L2 per step)",
                        "schedule": ("pipelined: step i+1's preparation beside step i's GEMM "
                                     "(two streams)") if args.pipeline else "serial",
+                       "amax": "given (reduced before the timed region)" if args.given_amax
+                               else "reduced in every call",
                        "parallelism": f"dp{world}"},
             "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
@@ -502,7 +512,8 @@ def run_gpu(args):
                      "bytes_per_elem": bpe,
                      "ms_in_step": prep_in_step,
                      "issue_roofline": issue,
-                     "kernel": " + ".join(prep_kernels(args.fmt, args.mask, args.residual)),
+                     "kernel": " + ".join(prep_kernels(args.fmt, args.mask, args.residual,
+                                                       args.given_amax)),
                      "note": "ms: calls back to back over input sets larger than L2 (X read "
                              "from HBM every call); ms_in_step: between events around the "
                              "call inside the step, which adds the first kernel's launch "
@@ -511,7 +522,8 @@ def run_gpu(args):
             "pct_fp4_peak": 100.0 * gemm_tflops / fp4_peak,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
                     "d2h_bytes_per_step": M * N * 2},
-            "gpu_launches": (len(prep_kernels(args.fmt, args.mask, args.residual)) + 1 +
+            "gpu_launches": (len(prep_kernels(args.fmt, args.mask, args.residual,
+                                              args.given_amax)) + 1 +
                              (1 if WS is not None else 0)) * args.steps,
             "clocks": clocks,
         }
@@ -680,6 +692,9 @@ def main():
     ap.add_argument("--pipeline", action="store_true",
                     help="two streams: the next step's (stack8b: group's) preparation runs "
                          "beside the current GEMM (sharq_prepare_alongside)")
+    ap.add_argument("--given-amax", action="store_true",
+                    help="NVFP4 pair mask: pass each input's tensor amax, reduced beforehand "
+                         "(sharq_prepare_given_amax), instead of reducing it in every call")
     ap.add_argument("--graph", action="store_true",
                     help="stack8b: replay the layers from one CUDA graph (no host calls in the "
                          "timed region)")

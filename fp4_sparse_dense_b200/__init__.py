@@ -22,11 +22,12 @@ from ._abi import (  # noqa: F401
     sharq_act_sizes, sharq_weight_sizes, sharq_status_string, sharq_device_status,
     sharq_prepare, sharq_quantize_weight, sharq_linear, sharq_linear_workspace_size,
     sharq_linear_noalloc, sharq_prepare_rmsnorm, sharq_wait_probe, sharq_prepare_alongside,
+    sharq_prepare_given_amax,
 )
 
 __all__ = [
     "Config", "QuantWeight", "PreparedAct", "quantize_weight", "prepare", "prepare_rmsnorm",
-    "linear", "sharq_prepare_rmsnorm", "sharq_prepare_alongside",
+    "linear", "sharq_prepare_rmsnorm", "sharq_prepare_alongside", "sharq_prepare_given_amax",
     "sharq_act_sizes", "sharq_weight_sizes", "sharq_prepare", "sharq_quantize_weight",
     "sharq_linear", "sharq_linear_workspace_size", "sharq_linear_noalloc", "sharq_device_status",
     "sharq_status_string", "SharqError", "linear_workspace",
@@ -154,14 +155,19 @@ def quantize_weight(W, cfg: Config = Config(), out: QuantWeight | None = None,
 
 
 def prepare(X, cfg: Config = Config(), out: PreparedAct | None = None, stream=None,
-            alongside: bool = False) -> PreparedAct:
+            alongside: bool = False, amax=None) -> PreparedAct:
     """X: CUDA tensor [M x K] (bf16/fp16) -> backbone / residual FP4 operands.
     alongside=True: launched to share the GPU with a GEMM running on another stream
-    (sharq_prepare_alongside; identical results)."""
+    (sharq_prepare_alongside; identical results). amax: a float32 CUDA tensor of one element,
+    the NVFP4 tensor amax to use instead of max |X| (sharq_prepare_given_amax)."""
     M, K = X.shape
     X = X.contiguous()
     out = out or empty_act(M, K, cfg, X.device)
     ca = out.c()
+    if amax is not None:
+        check(sharq_prepare_given_amax(_ptr(X), _dtype_code(X), _ptr(amax), ctypes.byref(ca),
+                                       _stream(stream)))
+        return out
     fn = sharq_prepare_alongside if alongside else sharq_prepare
     check(fn(_ptr(X), _dtype_code(X), ctypes.byref(ca), _stream(stream)))
     return out

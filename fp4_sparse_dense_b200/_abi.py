@@ -62,6 +62,7 @@ def _load():
         "sharq_quantize_weight": (st, [vp, ctypes.c_int, ctypes.POINTER(sharq_weight), vp]),
         "sharq_prepare": (st, [vp, ctypes.c_int, ctypes.POINTER(sharq_act), vp]),
         "sharq_prepare_alongside": (st, [vp, ctypes.c_int, ctypes.POINTER(sharq_act), vp]),
+        "sharq_prepare_given_amax": (st, [vp, ctypes.c_int, vp, ctypes.POINTER(sharq_act), vp]),
         "sharq_prepare_rmsnorm": (st, [vp, vp, ctypes.c_float, ctypes.c_int, vp,
                                        ctypes.POINTER(sharq_act), vp]),
         "sharq_linear": (st, [ctypes.POINTER(sharq_act), ctypes.POINTER(sharq_weight), vp,
@@ -87,6 +88,7 @@ sharq_weight_sizes = lib.sharq_weight_sizes
 sharq_quantize_weight = lib.sharq_quantize_weight
 sharq_prepare = lib.sharq_prepare
 sharq_prepare_alongside = lib.sharq_prepare_alongside
+sharq_prepare_given_amax = lib.sharq_prepare_given_amax
 sharq_prepare_rmsnorm = lib.sharq_prepare_rmsnorm
 sharq_linear = lib.sharq_linear
 sharq_linear_workspace_size = lib.sharq_linear_workspace_size

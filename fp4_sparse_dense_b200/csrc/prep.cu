@@ -373,7 +373,10 @@ __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
 // which is kept); byte permutes then keep the kept pairs' code bytes, either compressed
 // (the backbone operand) or in place with zeros elsewhere, which dequantise to the backbone
 // at kept positions and +0 elsewhere, so r = x - deq needs no per-element selection.
-template <bool BF16, int FMT, bool RESIDUAL, bool NORM, bool ABL>
+//
+// GIVEN (NVFP4): the tensor amax is supplied by the caller (p.amax_in), so this is the
+// only kernel of the call and it computes the mask itself.
+template <bool BF16, int FMT, bool RESIDUAL, bool NORM, bool ABL, bool GIVEN = false>
 __global__ void __launch_bounds__(256, ABL ? 1 : 3) prep_pair_kernel(PrepParams p) {
   constexpr bool NV = FMT == SHARQ_NVFP4;
   // ablation flags compile away unless ABL (the method's instantiation stays lean)
@@ -399,14 +402,16 @@ __global__ void __launch_bounds__(256, ABL ? 1 : 3) prep_pair_kernel(PrepParams 
   // after its own wait, so X is final here and the first item's load overlaps that kernel's
   // tail; the wait below returns once the mask kernel's writes (amax, metadata) are visible.
   // MXFP4 is the first kernel of the call: X may come from the kernel launched just before.
-  if (NV) wk.load(wk.first, row, q, cur);
+  if (NV && !GIVEN) wk.load(wk.first, row, q, cur);
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();  // the GEMM that follows may start its prologue
-  if (!NV) wk.load(wk.first, row, q, cur);
+  if (!NV || GIVEN) wk.load(wk.first, row, q, cur);
   AmaxState* const amax_st = reinterpret_cast<AmaxState*>(p.tensor_scale + 2);
   AmaxState* const amax_r_st = reinterpret_cast<AmaxState*>(p.tensor_scale + 4);
   if (NV && threadIdx.x == 0) {
-    if (res_phase == 2) {  // amax|X| as phase 1 wrote it; amax|r| from phase 1's reduction
+    if (GIVEN) {
+      s_amax = *p.amax_in;
+    } else if (res_phase == 2) {  // amax|X| as phase 1 wrote it; amax|r| from phase 1's reduction
       s_amax = *reinterpret_cast<volatile float*>(p.tensor_scale + 1);
       s_amax_r = __uint_as_float(*reinterpret_cast<volatile unsigned*>(&amax_r_st->acc));
     } else {
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(256, ABL ? 1 : 3) prep_pair_kernel(PrepParams 
   };
   // mask read back from bm (written by prep_mask_kernel, or supplied), else computed here
   // (MXFP4, and NVFP4 with RMSNorm absorbed, where the rstd kernel supplies the amax)
-  const bool meta_in = (NV && !(NORM && !ABL)) || mask_given;
+  const bool meta_in = (NV && !(NORM && !ABL) && !GIVEN) || mask_given;
   auto load_meta = [&](int it, int r, int q) -> uint32_t {
     if (!meta_in || it >= wk.n_items || r >= M) return 0x4444u;
     return __ldcg(reinterpret_cast<const unsigned short*>(wk.bm + wk.meta_off(q, r)));
@@ -616,7 +621,7 @@ __global__ void __launch_bounds__(256, ABL ? 1 : 3) prep_pair_kernel(PrepParams 
   }
   // NVFP4: the last CTA to finish resets the amax state it read for the next call (every
   // CTA read acc at its start; the fence orders that read before this CTA is counted)
-  if (NV && threadIdx.x == 0) {
+  if (NV && !GIVEN && threadIdx.x == 0) {
     AmaxState* const st = res_phase == 2 ? amax_r_st : amax_st;
     __threadfence();
     if (atomicAdd(&st->done, 1u) == gridDim.x - 1) {
@@ -835,6 +840,17 @@ static unsigned quant_threads(const PrepParams& p) { return p.alongside ? 128u :
 
 template <bool BF16, int FMT, bool RES, bool NORM, bool ABL>
 static cudaError_t launch_prep_t(const PrepParams& p, int mask, int num_sms, cudaStream_t st) {
+  if (FMT == SHARQ_NVFP4 && !NORM && !ABL && p.amax_in && is_pair_mask(mask)) {
+    // the caller's tensor amax: one kernel, mask computed inline
+    auto kern = prep_pair_kernel<BF16, FMT, RES, false, false, true>;
+    static int per_sm = 0;
+    unsigned blocks = 0;
+    const unsigned qt = quant_threads(p);
+    cudaError_t e = persistent_blocks(kern, &per_sm, p, num_sms, &blocks, qt);
+    if (e != cudaSuccess) return e;
+    if ((e = launch_pdl_t(kern, blocks, qt, p.alongside != 0, st, p)) != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   if (is_pair_mask(mask)) {
     cudaError_t e = cudaSuccess;
     // NVFP4 + RMSNorm (the method): the rstd kernel also reduces the tensor amax of the

@@ -229,7 +229,8 @@ namespace {
 // RMSNorm of X with (gamma, eps), writing the per-row rstd. alongside: launch sized to
 // share the SMs with a GEMM running on another stream (same results).
 sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, const void* gamma,
-                          float eps, float* rstd, void* stream, bool alongside = false) {
+                          float eps, float* rstd, void* stream, bool alongside = false,
+                          const float* amax_in = nullptr) {
   if (!X || !a) return SHARQ_ERR_INVALID_ARG;
   if (dtype != SHARQ_F16 && dtype != SHARQ_BF16) return SHARQ_ERR_INVALID_ARG;
   sharq_act_bytes sz;
@@ -239,6 +240,12 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
   const bool norm = gamma != nullptr;
   const bool pair = is_pair_mask(a->cfg.mask), none = a->cfg.mask == SHARQ_MASK_NONE;
   if (norm && !pair) return SHARQ_ERR_UNSUPPORTED;
+  // a supplied tensor amax: NVFP4, the method's pair mask, a residual with the shared s_g
+  // (or none), no RMSNorm
+  if (amax_in && ((reinterpret_cast<uintptr_t>(amax_in) & 3u) != 0)) return SHARQ_ERR_MISALIGNED;
+  if (amax_in && (a->cfg.fmt != SHARQ_NVFP4 || a->cfg.mask != SHARQ_MASK_PAIR_4_8 ||
+                  a->cfg.residual == 2 || a->cfg.residual == 3 || norm))
+    return SHARQ_ERR_UNSUPPORTED;
   // the pair-mask kernels address X and their outputs with 32-bit offsets
   if (pair && size_t(a->M) * size_t(a->K) >= (size_t(1) << 31)) return SHARQ_ERR_UNSUPPORTED;
   if (!a->bq || !a->bs || (!a->bm && !none) || !a->tensor_scale || (res && (!a->rq || !a->rs)) ||
@@ -285,6 +292,7 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
   p.res_unquant = a->cfg.residual == 2;
   p.alongside = alongside ? 1 : 0;
   p.res_phase = 0;
+  p.amax_in = amax_in;
   if (a->cfg.residual != 3)
     return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
   // the residual's own tensor scale: amax|r| is a grid-wide reduction that follows the
@@ -388,6 +396,12 @@ sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* a,
 sharq_status sharq_prepare_alongside(const void* X, sharq_dtype dtype, const sharq_act* a,
                                     void* stream) {
   return sharq::prepare_impl(X, dtype, a, nullptr, 0.f, nullptr, stream, true);
+}
+
+sharq_status sharq_prepare_given_amax(const void* X, sharq_dtype dtype, const float* amax,
+                                      const sharq_act* a, void* stream) {
+  if (!amax) return SHARQ_ERR_INVALID_ARG;
+  return sharq::prepare_impl(X, dtype, a, nullptr, 0.f, nullptr, stream, false, amax);
 }
 
 sharq_status sharq_prepare_rmsnorm(const void* X, const void* gamma, float eps, sharq_dtype dtype,

@@ -31,6 +31,7 @@ struct PrepParams {
   int res_unquant;      // residual against the unquantised backbone
   int alongside;        // launch sized to run beside a GEMM on another stream
   int res_phase;        // residual with its own tensor scale: 1 backbone + amax|r|, 2 residual
+  const float* amax_in; // NVFP4: the caller's tensor amax (device), else nullptr
 };
 
 struct WeightQuantParams {

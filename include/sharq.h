@@ -169,6 +169,18 @@ SHARQ_API sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, c
  * mask M * K must be below 2^31 (else SHARQ_ERR_UNSUPPORTED). */
 SHARQ_API sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* act, void* stream);
 
+/* The preparation with the NVFP4 tensor amax supplied by the caller instead of reduced from
+ * X in the call (a deployment option the SharQ page does not discuss: a static amax from
+ * calibration, or one a producer kernel has already reduced). amax: DEVICE pointer to one
+ * float (4-byte aligned), read by the kernel; s_g = amax / 2688 and every code, scale and
+ * metadata byte are those sharq_prepare would write if max |X| were that value (values of X
+ * above it saturate: E4M3 block scales clamp at 448, E2M1 codes at 6). With the amax known
+ * before X is read, the preparation is a single kernel that also computes the mask.
+ * NVFP4 with SHARQ_MASK_PAIR_4_8 and residual 0 or 1 only (else SHARQ_ERR_UNSUPPORTED);
+ * act->tensor_scale[0..1] receive s_g and amax as with sharq_prepare. */
+SHARQ_API sharq_status sharq_prepare_given_amax(const void* X, sharq_dtype dtype, const float* amax,
+                                    const sharq_act* act, void* stream);
+
 /* The same preparation, with results identical to sharq_prepare, launched to share the GPU
  * with a sharq_linear GEMM that runs at the same time on another stream (the overlap of
  * one batch's preparation with another batch's GEMM: the SharQ page's Fig. 4a latency
