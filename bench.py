@@ -435,20 +435,43 @@ def run_gpu(args):
     flops = 2.0 * M * N * K
     value = job_throughput(flops, world, args.steps, ms_max)
 
-    # end to end through the public API with host buffers (pinned), copies timed
+    # end to end through the public API with host buffers (pinned), copies timed: every step
+    # copies its X in and its Y out. The copies run on their own streams (one per
+    # direction, so PCIe carries both at once) and overlap the neighbouring steps' compute;
+    # a buffer set is reused only after the copy and the compute that use it are done.
     xh = [X[i].cpu().pin_memory() for i in range(n_sets)]
-    yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(1, min(args.steps, 10))
+    yh = [torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for _ in range(n_sets)]
+    e2e_steps = max(1, min(args.steps, 30))
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(n_sets)]
+    ev_done = [torch.cuda.Event() for _ in range(n_sets)]
+    ev_out = [torch.cuda.Event() for _ in range(n_sets)]
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
     for i in range(e2e_steps):
-        X[i % n_sets].copy_(xh[i % n_sets], non_blocking=True)
+        j = i % n_sets
+        with torch.cuda.stream(s_in):
+            if i >= n_sets:
+                s_in.wait_event(ev_done[j])  # step i - n_sets has read X[j]
+            X[j].copy_(xh[j], non_blocking=True)
+            ev_in[j].record(s_in)
+        stream.wait_event(ev_in[j])
+        if i >= n_sets:
+            stream.wait_event(ev_out[j])  # Y[j] of step i - n_sets has been copied out
         a = step(i)
-        sq.linear(a, QW[i % 2], out=Y[i % n_sets], workspace=WS)
-        yh.copy_(Y[i % n_sets], non_blocking=True)
+        sq.linear(a, QW[i % 2], out=Y[j], workspace=WS)
+        ev_done[j].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[j])
+            yh[j].copy_(Y[j], non_blocking=True)
+            ev_out[j].record(s_out)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_value = job_throughput(flops, world, e2e_steps,
