@@ -79,14 +79,36 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
-def _stream(stream):
+def _stream(stream, device=None):
+    """The cudaStream_t of `stream`, or of the current stream of `device` (a torch.device)."""
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
     torch = _torch()
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None and device is not None and device.index is not None:
+        return ctypes.c_void_p(raw(device.index))  # no Stream object per call
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+class _CStructCache:
+    """Caches the ctypes struct a buffer set passes to the C ABI; any field assignment
+    drops it, so the struct always holds the current buffers' addresses."""
+
+    def __setattr__(self, name, value):
+        if name != "_c":
+            self.__dict__.pop("_c", None)
+        object.__setattr__(self, name, value)
+
+    def c(self):
+        cs = self.__dict__.get("_c")
+        if cs is None:
+            cs = self._make_c()
+            self.__dict__["_c"] = cs
+        return cs
 
 
 @dataclass
-class QuantWeight:
+class QuantWeight(_CStructCache):
     codes: object
     scales_dense: object
     scales_sparse: object
@@ -95,13 +117,13 @@ class QuantWeight:
     N: int
     cfg: Config
 
-    def c(self) -> sharq_weight:
+    def _make_c(self) -> sharq_weight:
         return sharq_weight(_ptr(self.codes), _ptr(self.scales_dense), _ptr(self.scales_sparse),
                             _ptr(self.tensor_scale), self.K, self.N, self.cfg.c())
 
 
 @dataclass
-class PreparedAct:
+class PreparedAct(_CStructCache):
     bq: object
     bs: object
     bm: object
@@ -112,7 +134,7 @@ class PreparedAct:
     K: int
     cfg: Config
 
-    def c(self) -> sharq_act:
+    def _make_c(self) -> sharq_act:
         return sharq_act(_ptr(self.bq), _ptr(self.bs), _ptr(self.bm), _ptr(self.rq), _ptr(self.rs),
                          _ptr(self.tensor_scale), self.M, self.K, self.cfg.c())
 
@@ -161,15 +183,16 @@ def prepare(X, cfg: Config = Config(), out: PreparedAct | None = None, stream=No
     (sharq_prepare_alongside; identical results). amax: a float32 CUDA tensor of one element,
     the NVFP4 tensor amax to use instead of max |X| (sharq_prepare_given_amax)."""
     M, K = X.shape
-    X = X.contiguous()
+    if not X.is_contiguous():
+        X = X.contiguous()
     out = out or empty_act(M, K, cfg, X.device)
     ca = out.c()
     if amax is not None:
         check(sharq_prepare_given_amax(_ptr(X), _dtype_code(X), _ptr(amax), ctypes.byref(ca),
-                                       _stream(stream)))
+                                       _stream(stream, X.device)))
         return out
     fn = sharq_prepare_alongside if alongside else sharq_prepare
-    check(fn(_ptr(X), _dtype_code(X), ctypes.byref(ca), _stream(stream)))
+    check(fn(_ptr(X), _dtype_code(X), ctypes.byref(ca), _stream(stream, X.device)))
     return out
 
 
@@ -191,11 +214,18 @@ def prepare_rmsnorm(X, gamma, eps: float, cfg: Config = Config(), out: PreparedA
     return out, rstd
 
 
+_WS_BYTES = {}  # (M, N, K, cfg, device) -> bytes the shape's split-K wants
+
+
 def linear_workspace(M: int, N: int, K: int, cfg: Config = Config(), device="cuda"):
     """Caller-owned split-K workspace for sharq_linear (None when the shape does not split)."""
-    nbytes = ctypes.c_size_t(0)
-    check(sharq_linear_workspace_size(M, N, K, cfg.c(), ctypes.byref(nbytes)))
-    return _u8(nbytes.value, device) if nbytes.value else None
+    key = (M, N, K, cfg, str(device))
+    n = _WS_BYTES.get(key)
+    if n is None:
+        nbytes = ctypes.c_size_t(0)
+        check(sharq_linear_workspace_size(M, N, K, cfg.c(), ctypes.byref(nbytes)))
+        n = _WS_BYTES[key] = nbytes.value
+    return _u8(n, device) if n else None
 
 
 def linear(act: PreparedAct, w: QuantWeight, out=None, out_dtype=None, workspace="auto",
@@ -206,15 +236,19 @@ def linear(act: PreparedAct, w: QuantWeight, out=None, out_dtype=None, workspace
     caller may keep and pass again), None runs without splitting K, or a uint8 CUDA tensor.
     """
     torch = _torch()
-    out_dtype = out_dtype or torch.bfloat16
     if out is None:
-        out = torch.empty(act.M, w.N, dtype=out_dtype, device=act.bq.device)
-    code = {torch.bfloat16: BF16, torch.float32: F32}[out.dtype]
+        out = torch.empty(act.M, w.N, dtype=out_dtype or torch.bfloat16, device=act.bq.device)
+    if out.dtype == torch.bfloat16:
+        code = BF16
+    elif out.dtype == torch.float32:
+        code = F32
+    else:
+        raise TypeError(f"unsupported output dtype {out.dtype} (need bfloat16 or float32)")
     if isinstance(workspace, str):
         workspace = linear_workspace(act.M, w.N, act.K, act.cfg, act.bq.device)
     ws_ptr = _ptr(workspace)
     ws_bytes = workspace.numel() if workspace is not None else 0
     ca, cw = act.c(), w.c()
     check(sharq_linear(ctypes.byref(ca), ctypes.byref(cw), _ptr(out), code, ws_ptr, ws_bytes,
-                       _stream(stream)))
+                       _stream(stream, out.device)))
     return out
