@@ -166,7 +166,9 @@ SHARQ_API sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, c
  * mask the first pass also computes the mask and metadata, and the second reads them back;
  * the two kernels hand the tensor amax over through act->tensor_scale[2..3], so calls
  * that share one act->tensor_scale buffer must be ordered (one stream). With the pair
- * mask M * K must be below 2^31 (else SHARQ_ERR_UNSUPPORTED). */
+ * mask M * K must be below 2^31 (else SHARQ_ERR_UNSUPPORTED). X must be finite: an infinite
+ * or NaN element gives unspecified codes and scales (the kernels have no data-dependent
+ * control flow, so nothing faults or waits on it). */
 SHARQ_API sharq_status sharq_prepare(const void* X, sharq_dtype dtype, const sharq_act* act, void* stream);
 
 /* The preparation with the NVFP4 tensor amax supplied by the caller instead of reduced from
