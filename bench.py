@@ -557,6 +557,16 @@ def run_gpu(args):
                                             oracle_modes(args))
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores,
                                     "kind": "oracle", "sample": sample}
+            # the same oracle held to one thread (numpy's BLAS pool limited to 1)
+            try:
+                from threadpoolctl import threadpool_limits
+                with threadpool_limits(limits=1):
+                    v1, _, sample1 = cpu_baseline(args.workload, args.cpu_budget / 3, x16,
+                                                  qw_cpu, oracle_modes(args))
+                line["cpu_baseline"]["one_thread"] = {"value": v1, "unit": "TFLOP/s",
+                                                      "sample": sample1}
+            except ImportError:
+                pass
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
