@@ -79,10 +79,19 @@ def load_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and blank space (a comment edit leaves the code, and so
+    the kernels the counters were taken on, unchanged)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def src_hash(files):
     h = hashlib.sha1()
     for f in files:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
+        h.update(_code_only(open(os.path.join(ROOT, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:12]
 
 

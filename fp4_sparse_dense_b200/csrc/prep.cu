@@ -366,7 +366,8 @@ __global__ void __launch_bounds__(256) prep_mask_kernel(PrepParams p) {
 // current one. Scale and metadata bytes of neighbouring lanes are gathered with shuffles
 // into 32-bit stores, so no CTA barrier is needed inside the loop. NVFP4 runs after
 // prep_mask_kernel and takes the mask from its metadata and the tensor amax from its
-// reduction; MXFP4 needs no tensor scale and computes the mask inline.
+// reduction; MXFP4 (no tensor scale), NVFP4 with RMSNorm absorbed (the amax comes from the
+// rstd kernel) and NVFP4 with a supplied amax compute the mask inline.
 //
 // Per unit the backbone is encoded at all 32 positions with the block's scale (its max
 // |x| is the unit's max |x|: the largest element of every group of 8 lies in its top pair,
