@@ -1,0 +1,51 @@
+"""bench.py keeps its one-line JSON contract: a short run on the GPU prints exactly one JSON
+line with the keys the measurement needs (metric and value, the roofline of the dominant
+kernel with its traffic, the preparation's figures, the end-to-end number with the bytes
+it copies, the launch count and the clock record)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(*args):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "4",
+                          "--warmup", "3", "--no-cpu-baseline", *args],
+                         capture_output=True, text=True, cwd=ROOT, timeout=900)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+def test_bench_line_has_the_contract_keys():
+    d = _run()
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "roofline", "prep", "e2e", "gpu_launches", "clocks"):
+        assert k in d, k
+    assert d["steps"] == 4 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == "mlp_gate_up" and d["value"] > 0
+    r = d["roofline"]
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in r, k
+    assert r["bound"] == "tensor" and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+    assert r["traffic"] is not None  # the committed capture matches the current GEMM code
+    assert d["prep"]["issue_roofline"] is not None
+    e = d["e2e"]
+    assert e["h2d_bytes_per_step"] == 4096 * 4096 * 2 and e["d2h_bytes_per_step"] == 4096 * 14336 * 2
+    assert d["gpu_launches"] == 3 * 4  # mask, quantisation and GEMM per step
+    assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"]
+
+
+def test_bench_given_amax_mode():
+    d = _run("--given-amax")
+    assert d["prep"]["kernel"] == "prep_pair_kernel"
+    assert d["gpu_launches"] == 2 * 4
+    assert d["roofline"]["traffic"] is None  # the capture is of the default mode only
