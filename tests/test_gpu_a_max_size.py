@@ -40,7 +40,8 @@ def _rows_of_meta48(dev_buf, rows, Mp):
     return np.stack(out)
 
 
-def test_largest_accepted_tensor_prepare_and_linear():
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_largest_accepted_tensor_prepare_and_linear(fmt):
     import fp4_sparse_dense_b200 as sq
     import torch
     g = torch.Generator(device="cuda").manual_seed(2024)
@@ -49,7 +50,7 @@ def test_largest_accepted_tensor_prepare_and_linear():
         r1 = min(M, r0 + 8192)
         X[r0:r1] = (torch.randn(r1 - r0, K, generator=g, device="cuda") * 3).clamp_(-30, 30)
     X[PLANT] = 100.0
-    cfg = sq.Config()
+    cfg = sq.Config.from_names(fmt, "pair48", True)
     act = sq.prepare(X, cfg)
     rng = np.random.default_rng(9)
     w = gaussian_weight(rng, K, N)
@@ -58,20 +59,21 @@ def test_largest_accepted_tensor_prepare_and_linear():
     torch.cuda.synchronize()
     assert sq.sharq_device_status() == 0
 
-    amax = np.float32(100.0)
-    assert float(act.tensor_scale[0]) == S.tensor_scales(amax)[0]
+    amax = np.float32(100.0) if fmt == "nvfp4" else None
+    if fmt == "nvfp4":
+        assert float(act.tensor_scale[0]) == S.tensor_scales(amax)[0]
     rows = np.unique(np.concatenate([[0, 1, PLANT[0], M - 2, M - 1],
                                      rng.choice(M, 6, replace=False)]))
     xs = X[torch.from_numpy(rows).cuda()].float().cpu().numpy()
-    p = S.prepare(xs, "nvfp4", "pair48", amax=amax)
+    p = S.prepare(xs, fmt, "pair48", amax=amax)
     bq = act.bq.view(M, K // 4)[torch.from_numpy(rows).cuda()].cpu().numpy()
     rq = act.rq.view(M, K // 2)[torch.from_numpy(rows).cuda()].cpu().numpy()
     assert np.array_equal(bq, L.pack_nibbles(p.bq))
     assert np.array_equal(rq, L.pack_nibbles(p.rq))
     assert np.array_equal(_rows_of_scale_layout(act.bs, rows, K // 32), p.bs)
-    assert np.array_equal(_rows_of_scale_layout(act.rs, rows, K // 16), p.rs)
+    assert np.array_equal(_rows_of_scale_layout(act.rs, rows, K // S.residual_block(fmt)), p.rs)
     assert np.array_equal(_rows_of_meta48(act.bm, rows, (M + 127) // 128 * 128), p.meta)
 
-    y64 = S.linear(p, S.quantize_weight(w.values, "nvfp4", "pair48"))
+    y64 = S.linear(p, S.quantize_weight(w.values, fmt, "pair48"))
     ys = y[torch.from_numpy(rows).cuda()].double().cpu().numpy()
     assert rel_fro(ys, y64) <= 1e-5
