@@ -153,6 +153,25 @@ def test_prepare_rmsnorm_argument_checks(sq):
     assert f(p(0x1000), p(0x8000), 1e-6, sq.BF16, p(0x7000), ctypes.byref(elem), None) == 2
 
 
+def test_prepare_given_amax_and_alongside_argument_checks(sq):
+    p = ctypes.c_void_p
+    act = sq.sharq_act(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), p(0x6000),
+                       16, 256, sq.Config().c())
+    g = sq.sharq_prepare_given_amax
+    assert g(p(0x1000), sq.BF16, None, ctypes.byref(act), None) == 1  # no amax
+    assert g(p(0x1000), sq.BF16, p(0x7002), ctypes.byref(act), None) == 3  # misaligned amax
+    for names in (("mxfp4", "pair48", True), ("nvfp4", "elem24", True), ("nvfp4", "none", False),
+                  ("nvfp4", "pair48_given", True), ("nvfp4", "pair48", "own"),
+                  ("nvfp4", "pair48", "unquantized")):
+        other = sq.sharq_act(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), p(0x6000),
+                             16, 256, sq.Config.from_names(*names).c())
+        assert g(p(0x1000), sq.BF16, p(0x7000), ctypes.byref(other), None) == 2, names
+    a = sq.sharq_prepare_alongside
+    assert a(None, sq.BF16, ctypes.byref(act), None) == 1
+    assert a(p(0x1000), 7, ctypes.byref(act), None) == 1
+    assert a(p(0x1008), sq.BF16, ctypes.byref(act), None) == 3
+
+
 def test_wait_probe_argument_checks(sq):
     p = ctypes.c_void_p
     assert sq.sharq_wait_probe(None, 1, 10_000_000, None) == 1
