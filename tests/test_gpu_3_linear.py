@@ -182,6 +182,29 @@ def test_split_k_decode(M, K, N):
     check_y(y_bf16.float().cpu().numpy().astype(np.float64), y64, True)
 
 
+@pytest.mark.parametrize("out_f32", [True, False])
+def test_split_k_rows_independent_of_other_rows(out_f32):
+    """Split-K rows do not depend on the other rows of the call: rows 0..7 of a 16-row input
+    whose rows 8..15 are rows 0..7 halved (same tensor amax, so the same codes and scales
+    for rows 0..7, and the same K ranges, since both shapes have one row block) give Y
+    bit-identical to an 8-row call, the partials being summed in the same fixed order."""
+    import fp4_sparse_dense_b200 as sq
+    import torch
+    K, N = 14336, 4096
+    rng = np.random.default_rng(808)
+    x8 = to_device(heavy_activations(rng, 8, K, per_row=True))
+    x16 = torch.cat([x8, x8 * 0.5])
+    wt = sq.quantize_weight(to_device(gaussian_weight(rng, K, N)), cfg_of("nvfp4", "pair48"))
+    cfg = cfg_of("nvfp4", "pair48")
+    dt = torch.float32 if out_f32 else torch.bfloat16
+    y8 = sq.linear(sq.prepare(x8, cfg), wt, out_dtype=dt, workspace=sq.linear_workspace(8, N, K, cfg))
+    y16 = sq.linear(sq.prepare(x16, cfg), wt, out_dtype=dt,
+                    workspace=sq.linear_workspace(16, N, K, cfg))
+    torch.cuda.synchronize()
+    assert sq.sharq_device_status() == 0
+    assert torch.equal(y8, y16[:8])
+
+
 def test_split_k_workspace_reused_across_shapes():
     """One workspace, sized for the largest shape, serves several decode shapes in turn; each
     call's result is independent of what earlier calls left in it."""
