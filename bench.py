@@ -31,6 +31,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "SharQ linear TFLOPS (2MNK/t) and % FP4 peak; prep kernel HBM GB/s"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+NOMINAL_FP4_TFLOPS = 9000.0  # B200 dense FP4, spec sheet (context only)
+NOMINAL_HBM_GBS = 7700.0     # B200 HBM3e, HGX spec sheet (context only)
 L2_BYTES = 126 * 2**20  # B200 L2
 
 
@@ -538,9 +540,12 @@ def run_gpu(args):
                          "executed_frac": gemm_tflops / fp4_peak / metric_ceiling(args.mask, has_res),
                          # against 4x the measured bf16 burst figure instead of the sustained
                          "frac_vs_burst_peak": gemm_tflops / (bf16 * FP4_OVER_BF16),
+                         # context: the spec sheet's dense FP4 figure
+                         "frac_vs_nominal_peak": gemm_tflops / NOMINAL_FP4_TFLOPS,
                          "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg},
             "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
                      "frac": prep_gbs / hbm,
+                     "frac_vs_nominal_hbm": prep_gbs / NOMINAL_HBM_GBS,
                      "bytes_per_elem": bpe,
                      "ms_in_step": prep_in_step,
                      "issue_roofline": issue,
