@@ -234,14 +234,27 @@ def run_pipelined(n, slots, prep, gemm):
     main.wait_stream(side)
 
 
+def weight_bytes(qw):
+    """Bytes of a quantised weight the GEMM reads: codes and both scale views."""
+    return sum(b.numel() * b.element_size() for b in (qw.codes, qw.scales_dense, qw.scales_sparse)
+               if b is not None)
+
+
 def act_tensors(a):
     """The device buffers of a prepared activation (None where the configuration has none)."""
     return [t for t in (a.bq, a.bs, a.bm, a.rq, a.rs) if t is not None]
 
 
-def make_inputs(workload: str, seed: int):
+def workload_shape(args):
+    """(M, K, N) of a single-linear workload; --m replaces its token rows (decode sizes)."""
+    M, K, N, _ = WORKLOADS[args.workload]
+    return (args.m if args.m else M), K, N
+
+
+def make_inputs(workload: str, seed: int, M: int = None):
     from workloads import gaussian_weight, heavy_activations
-    M, K, N, per_row = WORKLOADS[workload]
+    M0, K, N, per_row = WORKLOADS[workload]
+    M = M or M0
     rng = np.random.default_rng(seed)
     x = heavy_activations(rng, M, K, per_row=per_row)
     w = gaussian_weight(rng, K, N)
@@ -264,7 +277,8 @@ def cpu_baseline(workload: str, budget_s: float, x, qw, kw=None):
     budget of CPU time is used. Returns (TFLOP/s, cores, sample description)."""
     from oracle import sharq as S
     kw = dict(kw or {})
-    M, K, N, _ = WORKLOADS[workload]
+    _, K, N, _ = WORKLOADS[workload]
+    M = x.values.shape[0]
     amax = S.amax_of(x.values) if kw.get("fmt", "nvfp4") == "nvfp4" else None
     given = None
     if kw.get("mask") == S.PAIR48_GIVEN:
@@ -277,7 +291,7 @@ def cpu_baseline(workload: str, budget_s: float, x, qw, kw=None):
         p = S.prepare(xs, amax=amax, given=None if given is None else given[: len(xs)], **kw)
         S.linear(p, qw)
         t_used += time.perf_counter() - t0
-        n_rows += rows
+        n_rows += len(xs)
     flops = 2.0 * n_rows * N * K
     cores = len(os.sched_getaffinity(0))
     return flops / t_used / 1e12, cores, f"{n_rows} of {M} rows x all {N} columns, K={K}; " \
@@ -292,8 +306,8 @@ def run_reference(args):
         raise SystemExit("the reference arm times the single-linear workloads "
                          f"({', '.join(WORKLOADS)})")
     from oracle import sharq as S
-    M, K, N, _ = WORKLOADS[args.workload]
-    x, w = make_inputs(args.workload, rank_seed(0))
+    M, K, N = workload_shape(args)
+    x, w = make_inputs(args.workload, rank_seed(0), M)
     kw = oracle_modes(args)
     qw = S.quantize_weight(w.values, args.fmt, args.mask)  # offline, outside the samples
     budget = max(1.0, 90.0 / max(1, args.steps + args.warmup))
@@ -333,17 +347,22 @@ def run_gpu(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     dev = torch.device("cuda", local)
-    M, K, N, _ = WORKLOADS[args.workload]
+    M, K, N = workload_shape(args)
     res_mode = {"on": True, "off": False, "unquantized": "unquantized", "own": "own"}[args.residual]
     cfg = sq.Config.from_names(args.fmt, args.mask, res_mode)  # default: the method
     has_res = args.residual != "off"
 
-    x16, w16 = make_inputs(args.workload, rank_seed(rank))
+    x16, w16 = make_inputs(args.workload, rank_seed(rank), M)
     from tests.gpu_helpers import to_device
     n_sets = 3
     X = [to_device(x16).to(dev) for _ in range(n_sets)]
     W = [to_device(w16).to(dev) for _ in range(2)]
     QW = [sq.quantize_weight(w, cfg) for w in W]
+    wbytes = weight_bytes(QW[0])
+    decode = M < 256  # the weight stream dominates: rotate enough copies to stream from HBM
+    if decode:
+        QW += [sq.quantize_weight(W[j % 2], cfg) for j in range(2, -(-int(2.5 * L2_BYTES) // wbytes))]
+    n_w = len(QW)
     ACT = [sq.empty_act(M, K, cfg, dev) for _ in range(n_sets)]
     Y = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(n_sets)]
     if args.mask == "pair48_given":
@@ -370,7 +389,7 @@ def run_gpu(args):
         return a
 
     for i in range(args.warmup):
-        sq.linear(step(i), QW[i % 2], out=Y[i % n_sets], workspace=WS)
+        sq.linear(step(i), QW[i % n_w], out=Y[i % n_sets], workspace=WS)
     torch.cuda.synchronize()
     status = sq.sharq_device_status()
     assert status == 0, sq.sharq_status_string(status)
@@ -385,11 +404,11 @@ def run_gpu(args):
             run_pipelined(k, n_sets,
                           lambda j, s: sq.prepare(X[j % n_sets], cfg, out=ACT[j % n_sets],
                                                   stream=s, alongside=True),
-                          lambda j: sq.linear(ACT[j % n_sets], QW[j % 2], out=Y[j % n_sets],
+                          lambda j: sq.linear(ACT[j % n_sets], QW[j % n_w], out=Y[j % n_sets],
                                               workspace=WS))
         else:
             for i in range(k):
-                sq.linear(step(i), QW[i % 2], out=Y[i % n_sets], workspace=WS)
+                sq.linear(step(i), QW[i % n_w], out=Y[i % n_sets], workspace=WS)
 
     if args.pipeline:  # warm the two-stream schedule too
         timed_steps(args.warmup)
@@ -414,7 +433,7 @@ def run_gpu(args):
         ev[i][0].record(stream)
         a = step(i)
         ev[i][1].record(stream)
-        sq.linear(a, QW[i % 2], out=Y[i % n_sets], workspace=WS)
+        sq.linear(a, QW[i % n_w], out=Y[i % n_sets], workspace=WS)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     prep_ms = [e[0].elapsed_time(e[1]) for e in ev]
@@ -424,6 +443,8 @@ def run_gpu(args):
     # behind the previous kernel) over enough input sets that every call reads X from HBM
     xb = M * K * 2 + sum(t.numel() * t.element_size() for t in act_tensors(ACT[0]))
     n_prep = max(2, -(-int(2.5 * L2_BYTES) // xb))
+    if decode:  # a few rows of X fit in L2 whatever we do; 64 sets bound the set-up
+        n_prep = min(n_prep, 64)
     XP = [X[j % n_sets] if j < n_sets else torch.empty_like(X[0]).copy_(X[j % n_sets])
           for j in range(n_prep)]
     AMP = [AMX[j % n_sets] for j in range(n_prep)]
@@ -475,7 +496,7 @@ def run_gpu(args):
         if i >= n_sets:
             stream.wait_event(ev_out[j])  # Y[j] of step i - n_sets has been copied out
         a = step(i)
-        sq.linear(a, QW[i % 2], out=Y[j], workspace=WS)
+        sq.linear(a, QW[i % n_w], out=Y[j], workspace=WS)
         ev_done[j].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[j])
@@ -501,7 +522,7 @@ def run_gpu(args):
         prep_gbs = M * K * bpe / (prep_avg * 1e-3) / 1e9
         # the committed capture is of the method's kernel (NVFP4, pair 4:8, residual on)
         method = ((args.fmt, args.mask, args.residual) == ("nvfp4", "pair48", "on")
-                  and not args.given_amax)
+                  and not args.given_amax and M == WORKLOADS[args.workload][0])
         traffic = traffic_from_profile(args.workload) if method else None
         clocks = clk.summary()
         # the preparation is bound by instruction issue, not HBM: its issue-rate roofline
@@ -523,7 +544,9 @@ def run_gpu(args):
             "data": "synthetic",
             "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": args.fmt,
                        "mask": args.mask, "residual": args.residual, "out": "bf16",
-                       "l2": f"{n_sets} rotating input sets (> 126 MB L2 per step)",
+                       "l2": (f"weights rotate over {n_w} copies ({n_w * wbytes / 1e6:.0f} MB "
+                              "> 126 MB L2)") if decode else
+                             f"{n_sets} rotating input sets (> 126 MB L2 per step)",
                        "schedule": ("pipelined: step i+1's preparation beside step i's GEMM "
                                     "(two streams)") if args.pipeline else "serial",
                        "amax": "given (reduced before the timed region)" if args.given_amax
@@ -551,10 +574,12 @@ def run_gpu(args):
                      "issue_roofline": issue,
                      "kernel": " + ".join(prep_kernels(args.fmt, args.mask, args.residual,
                                                        args.given_amax)),
-                     "note": "ms: calls back to back over input sets larger than L2 (X read "
-                             "from HBM every call); ms_in_step: between events around the "
-                             "call inside the step, which adds the first kernel's launch "
-                             "gap; algorithmic bytes count X once"},
+                     "note": ("ms: calls back to back over "
+                              + (f"{n_prep} input sets (a few rows: X stays in L2)" if decode
+                                 else "input sets larger than L2 (X read from HBM every call)")
+                              + "; ms_in_step: between events around the call inside the "
+                                "step, which adds the first kernel's launch gap; algorithmic "
+                                "bytes count X once")},
             "gemm_tflops": gemm_tflops,
             "pct_fp4_peak": 100.0 * gemm_tflops / fp4_peak,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
@@ -564,6 +589,15 @@ def run_gpu(args):
                              (1 if WS is not None else 0)) * args.steps,
             "clocks": clocks,
         }
+        if decode:  # below the ridge point the GEMM streams its weight: an HBM roofline
+            gbs = wbytes / (gemm_avg * 1e-3) / 1e9
+            line["roofline"] = {
+                "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "traffic": None, "peak_source": f"{peak_src}: copy bandwidth",
+                "note": "FP4 weight payload (codes and both scale views) / linear call time "
+                        "(split-K partials summed by a second kernel when the workspace is used)",
+                "weight_bytes": wbytes, "split_k": WS is not None,
+                "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg}
         if not args.no_cpu_baseline and world == 1:
             from oracle import sharq as S
             qw_cpu = S.quantize_weight(w16.values, args.fmt, args.mask)
@@ -599,7 +633,7 @@ def run_stack(args):
     from workloads import LLAMA8B_LINEARS
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
-    M = args.m
+    M = args.m or 1
     cfg = sq.Config.from_names(args.fmt, args.mask,
                                {"on": True, "off": False, "unquantized": "unquantized",
                                 "own": "own"}[args.residual])
@@ -732,7 +766,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
     ap.add_argument("--workload", default="mlp_gate_up", choices=list(WORKLOADS) + ["stack8b"])
-    ap.add_argument("--m", type=int, default=1, help="token rows of --workload stack8b")
+    ap.add_argument("--m", type=int, default=None,
+                    help="token rows: of --workload stack8b (default 1), or replacing a "
+                         "single-linear workload's M (decode sizes)")
     ap.add_argument("--fused", action="store_true",
                     help="stack8b: q|k|v and gate|up weights concatenated (4 GEMMs per layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

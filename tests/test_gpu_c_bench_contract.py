@@ -49,3 +49,16 @@ def test_bench_given_amax_mode():
     assert d["prep"]["kernel"] == "prep_pair_kernel"
     assert d["gpu_launches"] == 2 * 4
     assert d["roofline"]["traffic"] is None  # the capture is of the default mode only
+
+
+def test_bench_decode_rows():
+    """--m replaces a single-linear workload's token rows: below 256 rows the line's roofline
+    is the weight stream against HBM, the weights rotate over copies larger than L2, and
+    the split-K summing kernel is counted among the launches."""
+    d = _run("--workload", "mlp_down", "--m", "1")
+    assert d["config"]["M"] == 1 and d["config"]["workload"] == "mlp_down"
+    assert "copies" in d["config"]["l2"]
+    r = d["roofline"]
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["split_k"] is True
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+    assert d["gpu_launches"] == 4 * 4  # mask, quantisation, GEMM, split-K sum per step
