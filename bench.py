@@ -234,6 +234,15 @@ def run_pipelined(n, slots, prep, gemm):
     main.wait_stream(side)
 
 
+def input_sets(M: int, K: int, N: int) -> int:
+    """Input sets (X, its prepared buffers and Y) the timed steps rotate over: at least 3,
+    and enough that one rotation's X and Y exceed 2.5x the L2, so that no step finds its
+    operands in L2 from the previous rotation. Decode-sized M rotates its weights instead."""
+    if M < 256:
+        return 3
+    return max(3, -(-int(2.5 * L2_BYTES) // (M * K * 2 + M * N * 2)))
+
+
 def weight_bytes(qw):
     """Bytes of a quantised weight the GEMM reads: codes and both scale views."""
     return sum(b.numel() * b.element_size() for b in (qw.codes, qw.scales_dense, qw.scales_sparse)
@@ -354,7 +363,7 @@ def run_gpu(args):
 
     x16, w16 = make_inputs(args.workload, rank_seed(rank), M)
     from tests.gpu_helpers import to_device
-    n_sets = 3
+    n_sets = input_sets(M, K, N)
     X = [to_device(x16).to(dev) for _ in range(n_sets)]
     W = [to_device(w16).to(dev) for _ in range(2)]
     QW = [sq.quantize_weight(w, cfg) for w in W]
@@ -546,7 +555,8 @@ def run_gpu(args):
                        "mask": args.mask, "residual": args.residual, "out": "bf16",
                        "l2": (f"weights rotate over {n_w} copies ({n_w * wbytes / 1e6:.0f} MB "
                               "> 126 MB L2)") if decode else
-                             f"{n_sets} rotating input sets (> 126 MB L2 per step)",
+                             (f"{n_sets} rotating input sets ({n_sets * (M * K + M * N) * 2 / 1e6:.0f}"
+                              " MB of X and Y > 126 MB L2)"),
                        "schedule": ("pipelined: step i+1's preparation beside step i's GEMM "
                                     "(two streams)") if args.pipeline else "serial",
                        "amax": "given (reduced before the timed region)" if args.given_amax

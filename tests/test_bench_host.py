@@ -39,3 +39,11 @@ def test_cpu_baseline_counts_the_rows_it_ran(bench, M):
                                                "residual": True})
     assert sample.startswith(f"{M} of {M} rows")  # every row once, none counted twice
     assert value > 0 and cores >= 1
+
+
+def test_input_sets_exceed_l2(bench):
+    for M, K, N in [(4096, 4096, 14336), (2048, 4096, 4096), (4096, 14336, 4096), (256, 4096, 4096)]:
+        n = bench.input_sets(M, K, N)
+        assert n >= 3 and n * (M * K + M * N) * 2 >= 2.5 * bench.L2_BYTES
+    assert bench.input_sets(4096, 4096, 14336) == 3  # the default workload is unchanged
+    assert bench.input_sets(1, 14336, 4096) == 3     # decode rotates its weights instead
