@@ -585,8 +585,9 @@ def run_gpu(args):
                      "kernel": " + ".join(prep_kernels(args.fmt, args.mask, args.residual,
                                                        args.given_amax)),
                      "note": ("ms: calls back to back over "
-                              + (f"{n_prep} input sets (a few rows: X stays in L2)" if decode
-                                 else "input sets larger than L2 (X read from HBM every call)")
+                              + ("input sets larger than L2 (X read from HBM every call)"
+                                 if n_prep * xb >= 2 * L2_BYTES else
+                                 f"{n_prep} input sets (a few rows: X stays in L2)")
                               + "; ms_in_step: between events around the call inside the "
                                 "step, which adds the first kernel's launch gap; algorithmic "
                                 "bytes count X once")},
