@@ -362,10 +362,10 @@ def run_gpu(args):
     has_res = args.residual != "off"
 
     x16, w16 = make_inputs(args.workload, rank_seed(rank), M)
-    from tests.gpu_helpers import to_device
+    from workloads import to_device
     n_sets = input_sets(M, K, N)
-    X = [to_device(x16).to(dev) for _ in range(n_sets)]
-    W = [to_device(w16).to(dev) for _ in range(2)]
+    X = [to_device(x16, dev) for _ in range(n_sets)]
+    W = [to_device(w16, dev) for _ in range(2)]
     QW = [sq.quantize_weight(w, cfg) for w in W]
     wbytes = weight_bytes(QW[0])
     decode = M < 256  # the weight stream dominates: rotate enough copies to stream from HBM

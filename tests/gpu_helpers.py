@@ -6,17 +6,11 @@ import numpy as np
 
 from oracle import layouts as L
 from oracle import sharq as S
+from workloads import to_device  # noqa: F401  (re-exported for the tests)
 
 def torch_mod():
     import torch
     return torch
-
-
-def to_device(t16) -> "torch.Tensor":
-    """workloads.Tensor16 -> CUDA tensor of its 16-bit dtype, bit-identical."""
-    torch = torch_mod()
-    dt = torch.bfloat16 if t16.dtype == "bf16" else torch.float16
-    return torch.from_numpy(np.ascontiguousarray(t16.bits).view(np.int16).copy()).view(dt).cuda()
 
 
 def cfg_of(fmt: str, mask: str, residual: bool = True):

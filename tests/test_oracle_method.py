@@ -50,6 +50,91 @@ def test_worked_example_mxfp4():
     assert p.rs[0, 0] == e["rs_first"]
 
 
+GOLD_SG = os.path.join(os.path.dirname(__file__), "golden", "worked_block_nvfp4_sg_not_one.json")
+GOLD_W = os.path.join(os.path.dirname(__file__), "golden", "worked_weight_k64_n2.json")
+
+
+def test_worked_example_tensor_scale_not_one():
+    """s_g = float32(1.75 / 2688) != 1: the block scale comes from a * (448 / amax), where a
+    block max of 0.71875 lands exactly on an E4M3 tie (184 -> 192, code 0x74); the order
+    (a / 6) / s_g would give 0x73 (hand-worked fixture)."""
+    g = json.load(open(GOLD_SG))
+    x = np.zeros((1, 256), np.float32)
+    for k, v in g["x_nonzero"].items():
+        x[0, int(k)] = v
+    p = S.prepare(x, S.NVFP4, S.PAIR48)
+    e = g["expected"]
+    assert np.float32(p.s_g).view(np.uint32) == int(e["s_g_bits"], 16)
+    assert np.all(p.meta == e["meta_all"])
+    assert list(p.bq[0, :16]) == e["bq_block0"]
+    assert list(p.bq[0, 16:32]) == e["bq_block1"]
+    assert np.all(p.bq[0, 32:] == 0)
+    assert list(p.bs[0]) == e["bs"]
+    assert p.bs[0, 1] != e["bs_block1_other_order"]
+    assert list(p.rq[0, :48]) == e["rq_first48"]
+    assert np.all(p.rq[0, 48:] == 0)
+    assert list(p.rs[0]) == e["rs"]
+
+
+def _golden_w():
+    g = json.load(open(GOLD_W))
+    w = np.zeros((64, 2), np.float32)
+    for c, col in enumerate(("col0", "col1")):
+        for k, v in g["w_nonzero"][col].items():
+            w[int(k), c] = v
+    return g, w
+
+
+def _codes_match(wq_row, expect: dict):
+    want = np.zeros(wq_row.shape, np.uint8)
+    for k, v in expect.items():
+        want[int(k)] = v
+    return np.array_equal(wq_row, want)
+
+
+def test_worked_weight_pair_mask():
+    """Per-tensor amax (column 1's 0.5, not column 0's 0.25), 32-element blocks, the packed
+    payload and both scale views in the tiled layout (hand-worked fixture)."""
+    from oracle import layouts as L
+    g, w = _golden_w()
+    e = g["nvfp4_pair"]
+    qw = S.quantize_weight(w, S.NVFP4, S.PAIR48)
+    assert np.float32(qw.s_gw).view(np.uint32) == int(e["s_gw_bits"], 16)
+    assert qw.ws.tolist() == e["scales"]
+    assert _codes_match(qw.wq[0], e["codes_col0"]) and _codes_match(qw.wq[1], e["codes_col1"])
+    buf = S.weight_buffers(qw)
+    dense, sparse = buf["scales_dense"].reshape(-1), buf["scales_sparse"].reshape(-1)
+    assert dense.size == 512 and sparse.size == 512  # one 128 x 4 chunk each
+    assert list(dense[0:4]) == e["dense_view_row0"] and list(dense[16:20]) == e["dense_view_row1"]
+    assert list(sparse[0:4]) == e["sparse_view_row0"] and list(sparse[16:20]) == e["sparse_view_row1"]
+    rest = np.ones(512, bool)
+    rest[0:4] = rest[16:20] = False
+    assert not dense[rest].any() and not sparse[rest].any()
+    codes = buf["codes"].reshape(2, 32)
+    assert _codes_match(codes[0], e["packed_col0"]) and _codes_match(codes[1], e["packed_col1"])
+    assert L.pack_nibbles(qw.wq).shape == (2, 32)
+
+
+def test_worked_weight_16_element_blocks():
+    """NVFP4 without the pair mask quantises the weight in 16-element blocks: column 1's
+    second half-block gets its own scale and its K=20 value a different code."""
+    g, w = _golden_w()
+    e = g["nvfp4_16"]
+    qw = S.quantize_weight(w, S.NVFP4, S.ELEM24)
+    assert qw.ws.tolist() == e["scales"]
+    assert _codes_match(qw.wq[1], e["codes_col1"])
+    assert _codes_match(qw.wq[0], g["nvfp4_pair"]["codes_col0"])
+
+
+def test_worked_weight_mxfp4():
+    g, w = _golden_w()
+    e = g["mxfp4"]
+    qw = S.quantize_weight(w, S.MXFP4, S.PAIR48)
+    assert qw.s_gw == 1.0
+    assert qw.ws.tolist() == e["scales"]
+    assert _codes_match(qw.wq[0], e["codes_col0"]) and _codes_match(qw.wq[1], e["codes_col1"])
+
+
 # ----------------------------------------------------------------------------- masks
 
 

@@ -21,8 +21,7 @@ def _setup(M, K, N):
     import torch
 
     import fp4_sparse_dense_b200 as sq
-    from tests.gpu_helpers import to_device
-    from workloads import gaussian_weight, heavy_activations
+    from workloads import gaussian_weight, heavy_activations, to_device
     rng = np.random.default_rng(M + K + N)
     x = heavy_activations(rng, M, K, per_row=True)
     w = gaussian_weight(rng, K, N)

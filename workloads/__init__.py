@@ -78,6 +78,15 @@ class Tensor16:
         return self.values.shape
 
 
+def to_device(t16: Tensor16, device="cuda"):
+    """A Tensor16 as a torch tensor of its 16-bit dtype on `device`, bit-identical (the raw
+    patterns are reinterpreted, never converted). torch is imported only here."""
+    import torch
+    dt = torch.bfloat16 if t16.dtype == BF16 else torch.float16
+    bits = np.ascontiguousarray(t16.bits).view(np.int16).copy()
+    return torch.from_numpy(bits).view(dt).to(device)
+
+
 def _mk(x: np.ndarray, dtype: str) -> Tensor16:
     v, b = to_dtype(x, dtype)
     return Tensor16(v, b, dtype)
