@@ -1,15 +1,18 @@
 #!/usr/bin/env python
 """Benchmark of the SharQ sparse-dense FP4 linear layer on B200.
 
-One step = the whole hot path on one batch: activation preparation (tensor amax pass +
-fused mask / FP4 quantisation / residual / metadata kernel) and the fused sparse + dense
-FP4 GEMM with its bf16 epilogue. The weight is quantised once, before timing (it is an
-offline step). Inputs are seeded synthetic tensors with the workloads' shapes and value
-distributions (workloads/), resident in HBM before the timed region; several input sets
-rotate so that every step reads operands that are not in L2.
+One step = the whole hot path on one batch. The default workload is the 8B-shaped layer
+(the seven Llama-3-8B linears; q|k|v and gate|up concatenated along N, the deployment
+layout) at M = 8192 token rows: four activation preparations (tensor amax, pair mask, FP4
+backbone and residual, metadata) and four fused sparse + dense FP4 GEMMs with their bf16
+epilogues. Single linears (--workload mlp_gate_up / attn_proj / mlp_down) are the other
+workloads. Weights are quantised once, before timing (an offline step). Inputs are seeded
+synthetic tensors with the workloads' shapes and value distributions, resident in HBM
+before the timed region, and larger than L2 (or rotated so that no step finds its operands
+in L2).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mlp_gate_up]
-    python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload stack8b] [--m 8192]
+    python bench.py --impl reference ...   # the CPU oracle on bounded samples
 
 Multi-GPU (torchrun): every rank runs its own batch (independent token batches, no
 collective on the data path); value = all ranks' FLOPs / max-over-ranks time.
@@ -34,6 +37,7 @@ FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2
 NOMINAL_FP4_TFLOPS = 9000.0  # B200 dense FP4, spec sheet (context only)
 NOMINAL_HBM_GBS = 7700.0     # B200 HBM3e, HGX spec sheet (context only)
 L2_BYTES = 126 * 2**20  # B200 L2
+STACK_M = 8192  # default token rows of the 8B-shaped layer: the largest prefill of the sweep
 
 
 def prep_bytes_per_elem(fmt: str, mask: str, residual: bool) -> float:
@@ -81,6 +85,15 @@ def load_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def fp4_peak():
+    """Dense FP4 tensor peak for the GEMM roofline: 4 x the measured bf16 BURST figure (the
+    GEMM launches are timed as bursts at full clock; the sustained figure, taken at a lower
+    clock under the power cap, would flatter them). Returns (TFLOP/s, source)."""
+    _, bf16, bf16_sus, src = load_peaks()
+    return bf16 * FP4_OVER_BF16, (f"{src}: bf16 burst {bf16} x {FP4_OVER_BF16} (nominal FP4:BF16); "
+                                  f"context: x sustained {bf16_sus} = {bf16_sus * FP4_OVER_BF16:.1f}")
+
+
 def _code_only(text: str) -> str:
     """C++ source without comments and blank space (a comment edit leaves the code, and so
     the kernels the counters were taken on, unchanged)."""
@@ -110,7 +123,7 @@ def gemm_kernel_name(M: int, N: int, residual: str = "on") -> str:
 
 
 def traffic_from_profile(workload: str):
-    """DRAM bytes per GEMM launch from the committed ncu summary, when it was taken on the
+    """DRAM bytes per GEMM launch from the committed ncu record, when it was taken on the
     current GEMM source (else None)."""
     p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if not os.path.exists(p):
@@ -137,6 +150,18 @@ def prep_issue_from_profile(workload: str):
     if not e or e.get("prep_src") != src_hash(PREP_SRC):
         return None
     return e.get("warp_instructions_per_elem")
+
+
+def prep_traffic_from_profile(workload: str):
+    """DRAM bytes (read + write) per preparation call, all its kernels, from the committed
+    ncu record, when it was taken on the current preparation source (else None)."""
+    p = os.path.join(ROOT, "profiles", "prep_traffic.json")
+    if not os.path.exists(p):
+        return None
+    e = json.load(open(p)).get(workload)
+    if not e or e.get("prep_src") != src_hash(PREP_SRC):
+        return None
+    return e.get("dram_bytes_per_call")
 
 
 class Clocks:
@@ -307,33 +332,133 @@ def cpu_baseline(workload: str, budget_s: float, x, qw, kw=None):
         f"{t_used:.1f} s of CPU work (weight quantised beforehand)"
 
 
+# the 8B-shaped layer's CPU sample: rows of every linear's input x columns of its weight
+STACK_CPU_ROWS = 16
+STACK_CPU_COLS = 512
+
+
+def stack_layout(unfused: bool = False):
+    """Linears of the 8B-shaped layer: ({name: (K, N)}, [(group, K, [names])]), a group being
+    the linears that share one prepared input. Default: the deployment layout, q|k|v and
+    gate|up concatenated along N (four GEMMs); unfused: the seven linears."""
+    from workloads import LLAMA8B_LINEARS
+    if unfused:
+        shapes = {nm: (k, n) for nm, k, n in LLAMA8B_LINEARS}
+        groups = [("attn", 4096, ["q", "k", "v"]), ("o", 4096, ["o"]),
+                  ("mlp", 4096, ["gate", "up"]), ("down", 14336, ["down"])]
+    else:
+        shapes = {"qkv": (4096, 6144), "o": (4096, 4096), "gate_up": (4096, 28672),
+                  "down": (14336, 4096)}
+        groups = [("attn", 4096, ["qkv"]), ("o", 4096, ["o"]), ("mlp", 4096, ["gate_up"]),
+                  ("down", 14336, ["down"])]
+    return shapes, groups
+
+
+def stack_cpu_samples(shapes, groups, x_rows, amax_x, w_cols, amax_w, kw):
+    """Oracle operands of the layer's CPU sample: per linear the sampled input rows with the
+    input's tensor amax, and the weight's sampled columns quantised (offline, untimed) with
+    the weight's tensor amax. x_rows / amax_x are keyed by group, w_cols / amax_w by linear."""
+    from oracle import sharq as S
+    out = []
+    for gname, K, names in groups:
+        for nm in names:
+            qw = S.quantize_weight(w_cols[nm], kw.get("fmt", "nvfp4"), kw.get("mask", "pair48"),
+                                   amax=amax_w[nm])
+            out.append({"name": nm, "x": x_rows[gname], "amax": amax_x[gname], "qw": qw,
+                        "K": K, "cols": w_cols[nm].shape[1]})
+    return out
+
+
+def time_stack_passes(samples, budget_s, kw, min_passes=1):
+    """The oracle as it stands over the layer's sample (every linear: prepare the sampled rows,
+    multiply by the sampled weight columns), whole passes until the CPU-time budget is used.
+    Returns (TFLOP/s, passes, seconds, rows per linear)."""
+    from oracle import sharq as S
+    kw = dict(kw)
+    fmt = kw.get("fmt", "nvfp4")
+    t_used, flops, passes = 0.0, 0.0, 0
+    while passes < min_passes or t_used < budget_s:
+        for smp in samples:
+            t0 = time.perf_counter()
+            p = S.prepare(smp["x"], amax=smp["amax"] if fmt == "nvfp4" else None, **kw)
+            S.linear(p, smp["qw"])
+            t_used += time.perf_counter() - t0
+            flops += 2.0 * smp["x"].shape[0] * smp["cols"] * smp["K"]
+        passes += 1
+    return flops / t_used / 1e12, passes, t_used, samples[0]["x"].shape[0]
+
+
+def reference_stack_samples(args, rank_seed_: int):
+    """Synthetic sample of the 8B-shaped layer drawn on the host for the reference arm: the
+    workloads' generator (Student-t rows, 0.5 % outlier channels redrawn per row; W ~
+    N(0, 0.02)) for STACK_CPU_ROWS rows of every input and STACK_CPU_COLS columns of every
+    weight. The tensor amaxes are those of the drawn samples (the full tensors are not drawn)."""
+    from oracle import sharq as S
+    from workloads import gaussian_weight, heavy_activations
+    shapes, groups = stack_layout(args.unfused)
+    rng = np.random.default_rng(rank_seed_)
+    x_rows, amax_x, w_cols, amax_w = {}, {}, {}, {}
+    for gname, K, _ in groups:
+        x_rows[gname] = heavy_activations(rng, STACK_CPU_ROWS, K, per_row=True).values
+        amax_x[gname] = S.amax_of(x_rows[gname])
+    for nm, (k, n) in shapes.items():
+        w_cols[nm] = gaussian_weight(rng, k, STACK_CPU_COLS).values
+        amax_w[nm] = S.amax_of(w_cols[nm])
+    return stack_cpu_samples(shapes, groups, x_rows, amax_x, w_cols, amax_w, oracle_modes(args))
+
+
 def run_reference(args):
+    """The CPU oracle as it stands, timed on the host's cores on bounded samples of the same
+    workload (rank 0 only). Each step is one sample; ms_per_step is its real duration."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    if args.workload not in WORKLOADS:
-        raise SystemExit("the reference arm times the single-linear workloads "
-                         f"({', '.join(WORKLOADS)})")
     from oracle import sharq as S
-    M, K, N = workload_shape(args)
-    x, w = make_inputs(args.workload, rank_seed(0), M)
     kw = oracle_modes(args)
-    qw = S.quantize_weight(w.values, args.fmt, args.mask)  # offline, outside the samples
-    budget = max(1.0, 90.0 / max(1, args.steps + args.warmup))
-    for _ in range(args.warmup):
-        cpu_baseline(args.workload, budget, x, qw, kw)
-    vals = []
-    for _ in range(args.steps):
-        v, cores, sample = cpu_baseline(args.workload, budget, x, qw, kw)
-        vals.append(v)
+    cores = len(os.sched_getaffinity(0))
+    step_s, vals = [], []
+    if args.workload == "stack8b":
+        M = args.m or STACK_M
+        shapes, _ = stack_layout(args.unfused)
+        samples = reference_stack_samples(args, rank_seed(0))
+        for _ in range(args.warmup):
+            time_stack_passes(samples, 0.0, kw)
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            v, _, _, rows = time_stack_passes(samples, 0.0, kw)
+            step_s.append(time.perf_counter() - t0)
+            vals.append(v)
+        sample = (f"per step {rows} rows x {STACK_CPU_COLS} columns of each of the "
+                  f"{len(shapes)} linears ({', '.join(shapes)}), one pass; "
+                  f"{args.steps} steps, {sum(step_s):.1f} s of CPU work in total")
+        config = {"workload": "stack8b", "M": M, "fused": not args.unfused,
+                  "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
+                  "format": args.fmt, "mask": args.mask, "residual": args.residual}
+    else:
+        M, K, N = workload_shape(args)
+        x, w = make_inputs(args.workload, rank_seed(0), M)
+        qw = S.quantize_weight(w.values, args.fmt, args.mask)  # offline, outside the samples
+        budget = max(1.0, 90.0 / max(1, args.steps + args.warmup))
+        for _ in range(args.warmup):
+            cpu_baseline(args.workload, budget, x, qw, kw)
+        samples = []
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            v, cores, smp = cpu_baseline(args.workload, budget, x, qw, kw)
+            step_s.append(time.perf_counter() - t0)
+            vals.append(v)
+            samples.append(smp)
+        sample = (f"per step: {samples[0]}; {args.steps} steps, {sum(step_s):.1f} s of CPU "
+                  "work in total")
+        config = {"workload": args.workload, "M": M, "K": K, "N": N, "format": args.fmt,
+                  "mask": args.mask, "residual": args.residual}
     value = float(np.mean(vals))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 2.0 * M * N * K / (value * 1e12) * 1e3, "higher_is_better": True,
+        "ms_per_step": 1e3 * float(np.mean(step_s)), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": args.fmt,
-                   "mask": args.mask, "residual": args.residual},
+        "config": config,
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -343,19 +468,27 @@ def run_reference(args):
     return 0
 
 
-def run_gpu(args):
+def init_ranks():
+    """(world, rank, local, device, dist) of this process; NCCL group when world > 1."""
     import torch
     import torch.distributed as dist
-    import fp4_sparse_dense_b200 as sq
-
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
-    if world > 1:
+    if world > 1 and not dist.is_initialized():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    dev = torch.device("cuda", local)
+    return world, rank, local, torch.device("cuda", local), dist
+
+
+def run_gpu(args, emit: bool = True, light: bool = False):
+    """One single-linear workload. light: no end-to-end pass (used for the secondary line of
+    the default run). Returns the JSON line (rank 0) and prints it when emit."""
+    import torch
+    import fp4_sparse_dense_b200 as sq
+
+    world, rank, local, dev, dist = init_ranks()
     M, K, N = workload_shape(args)
     res_mode = {"on": True, "off": False, "unquantized": "unquantized", "own": "own"}[args.residual]
     cfg = sq.Config.from_names(args.fmt, args.mask, res_mode)  # default: the method
@@ -476,10 +609,47 @@ def run_gpu(args):
     flops = 2.0 * M * N * K
     value = job_throughput(flops, world, args.steps, ms_max)
 
-    # end to end through the public API with host buffers (pinned), copies timed: every step
-    # copies its X in and its Y out. The copies run on their own streams (one per
-    # direction, so PCIe carries both at once) and overlap the neighbouring steps' compute;
-    # a buffer set is reused only after the copy and the compute that use it are done.
+    e2e_value = None
+    if not light:
+        e2e_value = e2e_single(args, stream, X, Y, QW, WS, n_sets, n_w, step, flops, world, dist,
+                               dev)
+    line = None
+    if rank == 0:
+        line = single_line(args, world, M, K, N, n_sets, n_w, wbytes, decode, WS, flops, value,
+                           ms_max, gemm_ms, prep_b2b, prep_ms, n_prep, xb, e2e_value, clk, dev)
+        if not args.no_cpu_baseline and world == 1 and not light:
+            from oracle import sharq as S
+            qw_cpu = S.quantize_weight(w16.values, args.fmt, args.mask)
+            v, cores, sample = cpu_baseline(args.workload, args.cpu_budget, x16, qw_cpu,
+                                            oracle_modes(args))
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores,
+                                    "kind": "oracle", "sample": sample}
+            # the same oracle held to one thread (numpy's BLAS pool limited to 1)
+            try:
+                from threadpoolctl import threadpool_limits
+                with threadpool_limits(limits=1):
+                    v1, _, sample1 = cpu_baseline(args.workload, args.cpu_budget / 3, x16,
+                                                  qw_cpu, oracle_modes(args))
+                line["cpu_baseline"]["one_thread"] = {"value": v1, "unit": "TFLOP/s",
+                                                      "sample": sample1}
+            except ImportError:
+                pass
+        if emit:
+            print(json.dumps(line), flush=True)
+    if world > 1 and emit:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def e2e_single(args, stream, X, Y, QW, WS, n_sets, n_w, step, flops, world, dist, dev):
+    """End to end through the public API with host buffers (pinned), copies timed: every step
+    copies its X in and its Y out. The copies run on their own streams (one per direction,
+    so PCIe carries both at once) and overlap the neighbouring steps' compute; a buffer set
+    is reused only after the copy and the compute that use it are done."""
+    import torch
+    import fp4_sparse_dense_b200 as sq
+    M, N = Y[0].shape
     xh = [X[i].cpu().pin_memory() for i in range(n_sets)]
     yh = [torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for _ in range(n_sets)]
     e2e_steps = max(1, min(args.steps, 30))
@@ -519,10 +689,17 @@ def run_gpu(args):
                                max_over_ranks(e0.elapsed_time(e1), dist, dev))
     status = sq.sharq_device_status()
     assert status == 0, sq.sharq_status_string(status)
+    return e2e_value
 
-    if rank == 0:
+
+def single_line(args, world, M, K, N, n_sets, n_w, wbytes, decode, WS, flops, value, ms_max,
+                gemm_ms, prep_b2b, prep_ms, n_prep, xb, e2e_value, clk, dev):
+    """The JSON line of a single-linear workload (rank 0)."""
+    import torch
+    has_res = args.residual != "off"
+    if True:
         hbm, bf16, bf16_sus, peak_src = load_peaks()
-        fp4_peak = bf16_sus * FP4_OVER_BF16
+        peak, peak_source = fp4_peak()
         gemm_avg = float(np.mean(gemm_ms))
         prep_avg = prep_b2b
         prep_in_step = float(np.mean(prep_ms))
@@ -562,22 +739,21 @@ def run_gpu(args):
                        "amax": "given (reduced before the timed region)" if args.given_amax
                                else "reduced in every call",
                        "parallelism": f"dp{world}"},
-            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
-                         "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
+            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": gemm_tflops / peak,
                          "traffic": traffic,
-                         "peak_source": f"{peak_src}: bf16 sustained {bf16_sus} x "
-                                        f"{FP4_OVER_BF16} (nominal FP4:BF16)",
+                         "peak_source": peak_source,
                          "ceiling_frac": metric_ceiling(args.mask, has_res),
                          # the tensor pipe's executed work (sparse backbone at twice the
                          # dense rate): 2MNK / ceiling per launch, against the same peak
-                         "executed_frac": gemm_tflops / fp4_peak / metric_ceiling(args.mask, has_res),
-                         # against 4x the measured bf16 burst figure instead of the sustained
-                         "frac_vs_burst_peak": gemm_tflops / (bf16 * FP4_OVER_BF16),
-                         # context: the spec sheet's dense FP4 figure
+                         "executed_frac": gemm_tflops / peak / metric_ceiling(args.mask, has_res),
+                         # context: against 4x the sustained bf16 figure and the spec sheet
+                         "frac_vs_sustained_peak": gemm_tflops / (bf16_sus * FP4_OVER_BF16),
                          "frac_vs_nominal_peak": gemm_tflops / NOMINAL_FP4_TFLOPS,
                          "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg},
             "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
                      "frac": prep_gbs / hbm,
+                     "traffic": prep_traffic_from_profile(args.workload) if method else None,
                      "frac_vs_nominal_hbm": prep_gbs / NOMINAL_HBM_GBS,
                      "bytes_per_elem": bpe,
                      "ms_in_step": prep_in_step,
@@ -592,7 +768,7 @@ def run_gpu(args):
                                 "step, which adds the first kernel's launch gap; algorithmic "
                                 "bytes count X once")},
             "gemm_tflops": gemm_tflops,
-            "pct_fp4_peak": 100.0 * gemm_tflops / fp4_peak,
+            "pct_fp4_peak": 100.0 * gemm_tflops / peak,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
                     "d2h_bytes_per_step": M * N * 2},
             "gpu_launches": (len(prep_kernels(args.fmt, args.mask, args.residual,
@@ -609,85 +785,77 @@ def run_gpu(args):
                         "(split-K partials summed by a second kernel when the workspace is used)",
                 "weight_bytes": wbytes, "split_k": WS is not None,
                 "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg}
-        if not args.no_cpu_baseline and world == 1:
-            from oracle import sharq as S
-            qw_cpu = S.quantize_weight(w16.values, args.fmt, args.mask)
-            v, cores, sample = cpu_baseline(args.workload, args.cpu_budget, x16, qw_cpu,
-                                            oracle_modes(args))
-            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores,
-                                    "kind": "oracle", "sample": sample}
-            # the same oracle held to one thread (numpy's BLAS pool limited to 1)
-            try:
-                from threadpoolctl import threadpool_limits
-                with threadpool_limits(limits=1):
-                    v1, _, sample1 = cpu_baseline(args.workload, args.cpu_budget / 3, x16,
-                                                  qw_cpu, oracle_modes(args))
-                line["cpu_baseline"]["one_thread"] = {"value": v1, "unit": "TFLOP/s",
-                                                      "sample": sample1}
-            except ImportError:
-                pass
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+    return line
 
 
 def run_stack(args):
-    """One Llama-3-8B-shaped layer per step (config 5): q, k, v share one preparation of the
-    attention input, o has its own, gate and up share the MLP input's, down has its own.
-    Weights rotate over 4 layers (436 MB of FP4 payload), so a step streams its weights from
-    HBM as a model's would. Inputs are synthetic (drawn on the device, outlier channels per
-    row); they are not chained from layer to layer (there are no norms between them here)."""
+    """One Llama-3-8B-shaped layer per step: the attention input's preparation feeds q|k|v
+    (or q, k, v), o has its own, gate|up (or gate, up) share the MLP input's, down has its
+    own. Weights rotate over 4 layers (436 MB of FP4 payload), so a step streams its weights
+    from HBM as a model's would. Inputs are synthetic, drawn on the device: Student-t(4) rows
+    whose outlier channels (0.5 %, x U[20, 50]) are redrawn per row; they are not chained from
+    layer to layer (there are no norms between them here). Under torchrun every rank runs its
+    own batch (weak scaling)."""
     import torch
     import fp4_sparse_dense_b200 as sq
-    from workloads import LLAMA8B_LINEARS
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
-    M = args.m or 1
+    world, rank, local, dev, dist = init_ranks()
+    M = args.m or STACK_M
     cfg = sq.Config.from_names(args.fmt, args.mask,
                                {"on": True, "off": False, "unquantized": "unquantized",
                                 "own": "own"}[args.residual])
-    g = torch.Generator(device=dev).manual_seed(5000 + M)
-    shapes = {nm: (k, n) for nm, k, n in LLAMA8B_LINEARS}
-    groups = [("attn", 4096, ["q", "k", "v"]), ("o", 4096, ["o"]), ("mlp", 4096, ["gate", "up"]),
-              ("down", 14336, ["down"])]
-    if args.fused:  # deployment layout: q|k|v and gate|up weights concatenated along N
-        shapes = {"qkv": (4096, 6144), "o": (4096, 4096), "gate_up": (4096, 28672),
-                  "down": (14336, 4096)}
-        groups = [("attn", 4096, ["qkv"]), ("o", 4096, ["o"]), ("mlp", 4096, ["gate_up"]),
-                  ("down", 14336, ["down"])]
+    shapes, groups = stack_layout(args.unfused)
     layers = 4
+    g = torch.Generator(device=dev).manual_seed(5000 + M + 7919 * rank)
+    tdist = torch.distributions.StudentT(torch.tensor(4.0, device=dev))
 
-    def act_input(K):
-        x = torch.randn(M, K, device=dev, generator=g)
+    def act_input(K, idx):
+        # StudentT draws from the global stream: one seed per input
+        torch.manual_seed(5000 + M + 7919 * rank + 31 * idx)
+        x = tdist.sample((M, K))
         out = torch.rand(M, K, device=dev, generator=g) < 0.005
         gain = 20 + 30 * torch.rand(M, K, device=dev, generator=g)
         return torch.where(out, x * gain, x).to(torch.bfloat16)
 
-    X = {gname: act_input(K) for gname, K, _ in groups}
+    cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
+    if cpu:  # the CPU baseline (rank 0, one GPU): the oracle's own amax of every full tensor
+        from oracle import sharq as S
+    cols = {nm: np.linspace(0, n - 1, STACK_CPU_COLS).astype(np.int64)
+            for nm, (k, n) in shapes.items()}
+    w_cols, amax_w = {}, {}
+    X = {gname: act_input(K, i) for i, (gname, K, _) in enumerate(groups)}
     A = {gname: sq.empty_act(M, K, cfg, dev) for gname, K, _ in groups}
     QW = []
-    for _ in range(layers):
+    for li in range(layers):
         lw = {}
         for nm, (k, n) in shapes.items():
             w = (torch.randn(k, n, device=dev, generator=g) * 0.02).to(torch.bfloat16)
             lw[nm] = sq.quantize_weight(w, cfg)
+            if cpu and li == 0:  # the CPU baseline's weight sample (full-tensor amax)
+                w_cols[nm] = w[:, torch.from_numpy(cols[nm]).to(dev)].float().cpu().numpy()
+                amax_w[nm] = S.amax_of(w.float().cpu().numpy())
             del w
         QW.append(lw)
     Y = {nm: torch.empty(M, n, dtype=torch.bfloat16, device=dev) for nm, (k, n) in shapes.items()}
     WS = {nm: sq.linear_workspace(M, n, k, cfg, dev) for nm, (k, n) in shapes.items()}
     flops = sum(2.0 * M * k * n for k, n in shapes.values())
+    lin_flops = {nm: 2.0 * M * k * n for nm, (k, n) in shapes.items()}
     wbytes = 0
     for t in (QW[0][nm] for nm in shapes):
         wbytes += sum(b.numel() for b in (t.codes, t.scales_dense, t.scales_sparse) if b is not None)
+    stream = torch.cuda.current_stream()
 
-    def layer(i):
+    def layer(i, ev=None):
         lw = QW[i % layers]
         for gname, _, names in groups:
+            if ev is not None:
+                ev[gname][0].record(stream)
             a = sq.prepare(X[gname], cfg, out=A[gname])
+            if ev is not None:
+                ev[gname][1].record(stream)
             for nm in names:
                 sq.linear(a, lw[nm], out=Y[nm], workspace=WS[nm])
+                if ev is not None:
+                    ev[nm].record(stream)
 
     ng = len(groups)
 
@@ -723,8 +891,11 @@ def run_stack(args):
             graph.replay()
         torch.cuda.synchronize()
         assert sq.sharq_device_status() == 0
-    stream = torch.cuda.current_stream()
-    with Clocks(0) as clk:
+        stream = torch.cuda.current_stream()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         if graph is not None:
@@ -734,40 +905,239 @@ def run_stack(args):
             layers_run(args.steps)
         e1.record(stream)
         torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms, dist, dev)
     assert sq.sharq_device_status() == 0
-    per_layer_ms = ms / args.steps
-    hbm, bf16, bf16_sus, peak_src = load_peaks()
-    value = flops * args.steps / (ms * 1e-3) / 1e12
-    hbm_bound = M < 256  # weight stream dominates below the ridge point (~850 flop/byte)
-    achieved = (wbytes / (per_layer_ms * 1e-3) / 1e9) if hbm_bound else value
-    peak = hbm if hbm_bound else bf16_sus * FP4_OVER_BF16
-    n_prep = sum(len(prep_kernels(args.fmt, args.mask, args.residual)) for _ in groups)
-    n_gemm = sum(1 + (1 if WS[nm] is not None else 0) for nm in shapes)
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": per_layer_ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
-        "data": "synthetic (drawn on the device)",
-        "config": {"workload": "stack8b", "M": M, "fused": bool(args.fused),
-                   "schedule": "pipelined" if args.pipeline else "serial",
-                   "launch": f"CUDA graph of {layers} layers" if args.graph else "eager",
-                   "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
-                   "layers_rotated": layers, "format": args.fmt, "mask": args.mask,
-                   "residual": args.residual, "out": "bf16",
-                   "l2": f"weights rotate over {layers} layers ({layers * wbytes / 1e6:.0f} MB > 126 MB L2)",
-                   "parallelism": "dp1"},
-        "roofline": {"bound": "hbm" if hbm_bound else "tensor", "achieved": achieved, "peak": peak,
-                     "unit": "GB/s" if hbm_bound else "TFLOP/s", "frac": achieved / peak,
-                     "traffic": None,
-                     "note": ("FP4 weight payload (codes and both scale views) per layer / layer "
-                              "time" if hbm_bound else "2MNK of the 7 linears / layer time"),
-                     "weight_bytes_per_layer": wbytes},
-        "gpu_launches": (n_prep + n_gemm) * args.steps,
-        "clocks": clk.summary(),
-    }
-    print(json.dumps(line), flush=True)
+    if graph is not None:
+        del graph
+
+    # per-kernel durations: a second pass with events around every call on the launching
+    # stream (the first GEMM of a group then launches without its programmatic overlap)
+    n_ev = max(1, min(args.steps, 50))
+    evs = []
+    for i in range(n_ev):
+        ev = {gname: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for gname, _, _ in groups}
+        ev.update({nm: torch.cuda.Event(enable_timing=True) for nm in shapes})
+        layer(i, ev)
+        evs.append(ev)
+    torch.cuda.synchronize()
+    prep_ms = {gname: float(np.mean([e[gname][0].elapsed_time(e[gname][1]) for e in evs]))
+               for gname, _, _ in groups}
+    gemm_ms = {}
+    for gname, _, names in groups:
+        prev = [e[gname][1] for e in evs]
+        for nm in names:
+            gemm_ms[nm] = float(np.mean([p.elapsed_time(e[nm]) for p, e in zip(prev, evs)]))
+            prev = [e[nm] for e in evs]
+
+    # each preparation alone, calls back to back over copies of its input larger than L2
+    # together (X read from HBM every call)
+    prep_b2b = {}
+    for gname, K, _ in groups:
+        n_cp = max(2, -(-int(2.5 * L2_BYTES) // (M * K * 2)))
+        xs = [X[gname]] + [X[gname].clone() for _ in range(n_cp - 1)] if M >= 256 else [X[gname]]
+        for x in xs:
+            sq.prepare(x, cfg, out=A[gname])
+        torch.cuda.synchronize()
+        n_pc = max(3 * len(xs), 20)
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record(stream)
+        for j in range(n_pc):
+            sq.prepare(xs[j % len(xs)], cfg, out=A[gname])
+        p1.record(stream)
+        torch.cuda.synchronize()
+        prep_b2b[gname] = p0.elapsed_time(p1) / n_pc
+        del xs
+
+    e2e_value, h2d, d2h = e2e_stack(args, groups, shapes, X, Y, A, QW, WS, cfg, layers, flops,
+                                    world, dist, dev)
+    value = job_throughput(flops, world, args.steps, ms_max)
+
+    line = None
+    if rank == 0:
+        hbm, bf16, bf16_sus, peak_src = load_peaks()
+        clocks = clk.summary()
+        hbm_bound = M < 256  # weight stream dominates below the ridge point (~850 flop/byte)
+        has_res = args.residual != "off"
+        bpe = prep_bytes_per_elem(args.fmt, args.mask, has_res)
+        prep_bytes = sum(M * K * bpe for _, K, _ in groups)
+        prep_time = sum(prep_b2b.values())
+        gemm_time = sum(gemm_ms.values())
+        gemm_tflops = flops / (gemm_time * 1e-3) / 1e12
+        method = ((args.fmt, args.mask, args.residual) == ("nvfp4", "pair48", "on")
+                  and not args.unfused and M == STACK_M)
+        key = f"stack8b_m{M}"
+        launches = [{"linear": nm, "M": M, "K": k, "N": n, "ms": gemm_ms[nm],
+                     "tflops": lin_flops[nm] / (gemm_ms[nm] * 1e-3) / 1e12,
+                     "kernel": gemm_kernel_name(M, n, args.residual)}
+                    for nm, (k, n) in shapes.items()]
+        if hbm_bound:
+            achieved = wbytes / (gemm_time * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "traffic": None,
+                    "peak_source": f"{peak_src}: copy bandwidth",
+                    "note": "FP4 weight payload (codes and both scale views) of the layer / the "
+                            "layer's linear call times (GEMM and split-K sum)",
+                    "weight_bytes_per_layer": wbytes, "launches": launches}
+        else:
+            peak, peak_source = fp4_peak()
+            roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s",
+                    "frac": gemm_tflops / peak,
+                    "traffic": traffic_from_profile(key) if method else None,
+                    "traffic_scope": "DRAM bytes per GEMM launch, mean over the layer's "
+                                     f"{len(shapes)} launches",
+                    "peak_source": peak_source,
+                    "ceiling_frac": metric_ceiling(args.mask, has_res),
+                    "executed_frac": gemm_tflops / peak / metric_ceiling(args.mask, has_res),
+                    "frac_vs_sustained_peak": gemm_tflops / (bf16_sus * FP4_OVER_BF16),
+                    "frac_vs_nominal_peak": gemm_tflops / NOMINAL_FP4_TFLOPS,
+                    "note": "2MNK of the layer's linears / the sum of their GEMM launches' "
+                            "mean durations (events around each call on the launching stream)",
+                    "kernel": gemm_kernel_name(M, 4096, args.residual), "launches": launches}
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
+            "data": "synthetic (drawn on the device: Student-t(4) rows, 0.5 % outlier channels "
+                    "x U[20,50] redrawn per row; W ~ N(0, 0.02), random init)",
+            "config": {"workload": "stack8b", "M": M, "fused": not args.unfused,
+                       "schedule": "pipelined" if args.pipeline else "serial",
+                       "launch": f"CUDA graph of {layers} layers" if args.graph else "eager",
+                       "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
+                       "layers_rotated": layers, "format": args.fmt, "mask": args.mask,
+                       "residual": args.residual, "out": "bf16",
+                       "l2": (f"weights rotate over {layers} layers ({layers * wbytes / 1e6:.0f} MB"
+                              f"); X {sum(M * K * 2 for _, K, _ in groups) / 1e6:.0f} MB and Y "
+                              f"{sum(M * n * 2 for _, n in shapes.values()) / 1e6:.0f} MB per "
+                              "layer" + (" (inputs larger than the 126 MB L2)" if M >= 4096
+                                         else "")),
+                       "parallelism": f"dp{world}"},
+            "roofline": roof,
+            "prep": {"ms": prep_time, "gbs": prep_bytes / (prep_time * 1e-3) / 1e9,
+                     "hbm_peak_gbs": hbm, "frac": prep_bytes / (prep_time * 1e-3) / 1e9 / hbm,
+                     "traffic": prep_traffic_from_profile(key) if method else None,
+                     "traffic_scope": "DRAM bytes per preparation call, mean over the layer's "
+                                      f"{len(groups)} calls",
+                     "bytes_per_elem": bpe, "ms_in_step": sum(prep_ms.values()),
+                     "calls": [{"input": gname, "M": M, "K": K, "ms": prep_b2b[gname],
+                                "gbs": M * K * bpe / (prep_b2b[gname] * 1e-3) / 1e9}
+                               for gname, K, _ in groups],
+                     "kernel": " + ".join(prep_kernels(args.fmt, args.mask, args.residual)),
+                     "note": "ms: the layer's preparation calls, each timed back to back over "
+                             "copies of its input larger than L2 (X from HBM every call); "
+                             "ms_in_step: between events around the calls inside the step"},
+            "gemm_tflops": gemm_tflops,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": (sum(len(prep_kernels(args.fmt, args.mask, args.residual))
+                                 for _ in groups)
+                             + sum(1 + (1 if WS[nm] is not None else 0) for nm in shapes))
+                            * args.steps,
+            "clocks": clocks,
+        }
+    # release the layer's buffers before the secondary workload and the CPU baseline
+    x_rows, amax_x = {}, {}
+    if cpu:
+        rows = np.linspace(0, M - 1, min(M, STACK_CPU_ROWS)).astype(np.int64)
+        for gname, _, _ in groups:
+            xh = X[gname].float().cpu().numpy()
+            x_rows[gname] = np.ascontiguousarray(xh[rows])
+            amax_x[gname] = S.amax_of(xh)
+            del xh
+    del X, A, QW, Y, WS
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_secondary and M == STACK_M:
+        sub = argparse.Namespace(**vars(args))
+        sub.workload, sub.m, sub.steps = "mlp_gate_up", None, min(args.steps, 200)
+        sub.no_cpu_baseline, sub.pipeline, sub.given_amax = True, False, False
+        d = run_gpu(sub, emit=False, light=True)
+        line["secondary"] = [{
+            "workload": "mlp_gate_up", "M": 4096, "K": 4096, "N": 14336,
+            "value": d["value"], "unit": "TFLOP/s", "steps": sub.steps,
+            "gemm_tflops": d["roofline"]["achieved"], "gemm_frac": d["roofline"]["frac"],
+            "gemm_traffic": d["roofline"]["traffic"], "prep_gbs": d["prep"]["gbs"],
+            "prep_frac": d["prep"]["frac"], "prep_traffic": d["prep"]["traffic"],
+            "clocks": d["clocks"]}]
+    if cpu:
+        samples = stack_cpu_samples(shapes, groups, x_rows, amax_x, w_cols, amax_w,
+                                    oracle_modes(args))
+        v, passes, t_used, nrows = time_stack_passes(samples, args.cpu_budget, oracle_modes(args))
+        line["cpu_baseline"] = {
+            "value": v, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"{nrows} of {M} rows x {STACK_CPU_COLS} columns of each of the "
+                      f"{len(shapes)} linears ({', '.join(shapes)}), {passes} passes, "
+                      f"{t_used:.1f} s of CPU work; the weights' sampled columns quantised "
+                      "beforehand with each full tensor's amax, the rows prepared with each "
+                      "full input's amax"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
     return 0
+
+
+def e2e_stack(args, groups, shapes, X, Y, A, QW, WS, cfg, layers, flops, world, dist, dev):
+    """End to end through the public API with host buffers: every step copies the layer's
+    inputs in from pinned memory and its outputs out, on one copy stream per direction that
+    overlaps the neighbouring steps' compute (two buffer sets). Returns (TFLOP/s, bytes in,
+    bytes out per step)."""
+    import torch
+    import fp4_sparse_dense_b200 as sq
+    n_sets = 2
+    stream = torch.cuda.current_stream()
+    Xd = [X] + [{k: torch.empty_like(v) for k, v in X.items()} for _ in range(n_sets - 1)]
+    Yd = [Y] + [{k: torch.empty_like(v) for k, v in Y.items()} for _ in range(n_sets - 1)]
+    xh = [{k: v.cpu().pin_memory() for k, v in X.items()} for _ in range(n_sets)]
+    yh = [{k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in Y.items()}
+          for _ in range(n_sets)]
+    h2d = sum(v.numel() * 2 for v in X.values())
+    d2h = sum(v.numel() * 2 for v in Y.values())
+    steps = max(1, min(args.steps, 20))
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(n_sets)]
+    ev_done = [torch.cuda.Event() for _ in range(n_sets)]
+    ev_out = [torch.cuda.Event() for _ in range(n_sets)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    for i in range(steps):
+        j = i % n_sets
+        with torch.cuda.stream(s_in):
+            if i >= n_sets:
+                s_in.wait_event(ev_done[j])  # step i - n_sets has read these inputs
+            for k in Xd[j]:
+                Xd[j][k].copy_(xh[j][k], non_blocking=True)
+            ev_in[j].record(s_in)
+        stream.wait_event(ev_in[j])
+        if i >= n_sets:
+            stream.wait_event(ev_out[j])  # the outputs of step i - n_sets have been copied out
+        lw = QW[i % layers]
+        for gname, _, names in groups:
+            a = sq.prepare(Xd[j][gname], cfg, out=A[gname])
+            for nm in names:
+                sq.linear(a, lw[nm], out=Yd[j][nm], workspace=WS[nm])
+        ev_done[j].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[j])
+            for k in Yd[j]:
+                yh[j][k].copy_(Yd[j][k], non_blocking=True)
+            ev_out[j].record(s_out)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    value = job_throughput(flops, world, steps, max_over_ranks(e0.elapsed_time(e1), dist, dev))
+    assert sq.sharq_device_status() == 0
+    return value, h2d, d2h
 
 
 def main():
@@ -776,13 +1146,18 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
-    ap.add_argument("--workload", default="mlp_gate_up", choices=list(WORKLOADS) + ["stack8b"])
+    ap.add_argument("--workload", default="stack8b", choices=["stack8b"] + list(WORKLOADS),
+                    help="stack8b: the 8B-shaped layer (default, M = 8192); the others are "
+                         "single linears")
     ap.add_argument("--m", type=int, default=None,
-                    help="token rows: of --workload stack8b (default 1), or replacing a "
-                         "single-linear workload's M (decode sizes)")
-    ap.add_argument("--fused", action="store_true",
-                    help="stack8b: q|k|v and gate|up weights concatenated (4 GEMMs per layer)")
+                    help=f"token rows: of --workload stack8b (default {STACK_M}), or replacing "
+                         "a single-linear workload's M (decode sizes)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="stack8b: the seven linears as separate GEMMs (default: q|k|v and "
+                         "gate|up weights concatenated along N, four GEMMs per layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="stack8b at the default M: skip the mlp_gate_up figures added to the line")
     ap.add_argument("--pipeline", action="store_true",
                     help="two streams: the next step's (stack8b: group's) preparation runs "
                          "beside the current GEMM (sharq_prepare_alongside)")
@@ -806,8 +1181,12 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
     if args.workload == "stack8b":
+        if args.given_amax or args.mask == "pair48_given":
+            raise SystemExit("stack8b runs the method's preparation (no --given-amax, no "
+                             "supplied mask)")
         return run_stack(args)
-    return run_gpu(args)
+    run_gpu(args)
+    return 0
 
 
 if __name__ == "__main__":

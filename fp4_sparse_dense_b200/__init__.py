@@ -20,6 +20,7 @@ from ._abi import (  # noqa: F401
     lib_path,
     sharq_act, sharq_act_bytes, sharq_config, sharq_weight, sharq_weight_bytes, check,
     sharq_act_sizes, sharq_weight_sizes, sharq_status_string, sharq_device_status,
+    sharq_read_device_status,
     sharq_prepare, sharq_quantize_weight, sharq_linear, sharq_linear_workspace_size,
     sharq_linear_noalloc, sharq_prepare_rmsnorm, sharq_wait_probe, sharq_prepare_alongside,
     sharq_prepare_given_amax,
@@ -30,6 +31,7 @@ __all__ = [
     "linear", "sharq_prepare_rmsnorm", "sharq_prepare_alongside", "sharq_prepare_given_amax",
     "sharq_act_sizes", "sharq_weight_sizes", "sharq_prepare", "sharq_quantize_weight",
     "sharq_linear", "sharq_linear_workspace_size", "sharq_linear_noalloc", "sharq_device_status",
+    "sharq_read_device_status",
     "sharq_status_string", "SharqError", "linear_workspace",
     "NVFP4", "MXFP4", "PAIR_4_8", "ELEM_2_4", "F16", "BF16", "F32",
 ]

@@ -72,6 +72,7 @@ def _load():
         "sharq_linear_noalloc": (st, [ctypes.POINTER(sharq_act), ctypes.POINTER(sharq_weight),
                                       vp, ctypes.c_int, vp]),
         "sharq_device_status": (st, []),
+        "sharq_read_device_status": (st, [vp]),
         "sharq_wait_probe": (st, [vp, ctypes.c_uint32, ctypes.c_uint64, vp]),
         "sharq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
@@ -94,6 +95,7 @@ sharq_linear = lib.sharq_linear
 sharq_linear_workspace_size = lib.sharq_linear_workspace_size
 sharq_linear_noalloc = lib.sharq_linear_noalloc
 sharq_device_status = lib.sharq_device_status
+sharq_read_device_status = lib.sharq_read_device_status
 sharq_wait_probe = lib.sharq_wait_probe
 sharq_status_string = lib.sharq_status_string
 

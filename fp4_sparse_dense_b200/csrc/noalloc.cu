@@ -28,15 +28,18 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_scratch_mu;
-std::unordered_map<int, void*> g_scratch_addr;  // device ordinal -> device address
+// context id -> device address of the array in that context. A device reset creates a new
+// primary context with a new id, so an address from before the reset is never reused.
+std::unordered_map<unsigned long long, void*> g_scratch_addr;
 
-// Device address of the scratch on the current device; looked up on the first call per
-// device (with that device current) and cached.
+// Device address of the scratch in the current context; looked up with
+// cudaGetSymbolAddress on the first call in each context (with that device current) and
+// cached.
 sharq_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SHARQ_ERR_CUDA;
+  unsigned long long ctx = 0;
+  if (current_context_id(&ctx) != SHARQ_OK) return SHARQ_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  auto it = g_scratch_addr.find(dev);
+  auto it = g_scratch_addr.find(ctx);
   if (it != g_scratch_addr.end()) {
     *out = it->second;
     return SHARQ_OK;
@@ -44,7 +47,7 @@ sharq_status scratch_address(void** out) {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
     return SHARQ_ERR_CUDA;
-  g_scratch_addr[dev] = p;
+  g_scratch_addr[ctx] = p;
   *out = p;
   return SHARQ_OK;
 }

@@ -13,9 +13,46 @@
 
 namespace sharq {
 
-// Written by kernels that give up on a bounded wait; read and cleared by
-// sharq_device_status(). One word per device (the array is per device image).
-__device__ unsigned int g_status_word;
+// Unique id of the calling thread's current CUDA context (CUDA 12 context ids are never
+// reused within a process, unlike context handles, so caches keyed on them are not fooled
+// by a device reset that creates a new primary context). Initialises the device's primary
+// context if none is current.
+sharq_status current_context_id(unsigned long long* id) {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  if (!get_current || !get_id) return SHARQ_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return SHARQ_ERR_CUDA;
+  if (!ctx) {  // no context yet: cudaSetDevice initialises the device's primary context
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess ||
+        get_current(&ctx) != CUDA_SUCCESS || !ctx)
+      return SHARQ_ERR_CUDA;
+  }
+  return get_id(ctx, id) == CUDA_SUCCESS ? SHARQ_OK : SHARQ_ERR_CUDA;
+}
+
+// Status words written by kernels that give up on a bounded wait: one word per stream
+// slot (a stream's launches report to its slot), read and cleared by
+// sharq_read_device_status (the stream's slot, in stream order) and sharq_device_status
+// (every slot, after a device synchronisation). The arrays are per device image.
+constexpr int kStatusSlots = 64;
+__device__ unsigned int g_status_words[kStatusSlots];
+__device__ unsigned int g_status_taken[kStatusSlots + 1];  // [kStatusSlots]: all slots
 
 namespace {
 
@@ -24,22 +61,39 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per mbarrier 
 struct DeviceInfo {
   bool ok = false;
   int num_sms = 0;
-  unsigned int* status = nullptr;
+  unsigned long long ctx_id = 0;
+  unsigned int* status_words = nullptr;  // device addresses of the arrays above
+  unsigned int* status_taken = nullptr;
 };
 
 std::mutex g_mu;
-std::unordered_map<int, DeviceInfo> g_dev;
+std::unordered_map<unsigned long long, DeviceInfo> g_dev;  // context id -> device facts
+struct StreamKey {
+  unsigned long long ctx;
+  const void* stream;
+  bool operator==(const StreamKey& o) const { return ctx == o.ctx && stream == o.stream; }
+};
+struct StreamKeyHash {
+  size_t operator()(const StreamKey& k) const {
+    return size_t(k.ctx * 0x9E3779B97F4A7C15ull) ^ reinterpret_cast<size_t>(k.stream);
+  }
+};
+std::unordered_map<StreamKey, int, StreamKeyHash> g_stream_slot;
+std::unordered_map<unsigned long long, int> g_next_slot;  // context id -> next slot to hand out
 
 sharq_status device_info(DeviceInfo* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SHARQ_ERR_CUDA;
+  unsigned long long ctx = 0;
+  if (current_context_id(&ctx) != SHARQ_OK) return SHARQ_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  auto it = g_dev.find(dev);
+  auto it = g_dev.find(ctx);
   if (it != g_dev.end()) {
     *out = it->second;
     return out->ok ? SHARQ_OK : SHARQ_ERR_ARCH;
   }
   DeviceInfo d;
+  d.ctx_id = ctx;
   int major = 0, minor = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -47,13 +101,37 @@ sharq_status device_info(DeviceInfo* out) {
     return SHARQ_ERR_CUDA;
   d.ok = (major == 10 && minor == 0);
   if (d.ok) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return SHARQ_ERR_CUDA;
-    d.status = static_cast<unsigned int*>(p);
+    void* w = nullptr;
+    void* t = nullptr;
+    if (cudaGetSymbolAddress(&w, g_status_words) != cudaSuccess ||
+        cudaGetSymbolAddress(&t, g_status_taken) != cudaSuccess)
+      return SHARQ_ERR_CUDA;
+    d.status_words = static_cast<unsigned int*>(w);
+    d.status_taken = static_cast<unsigned int*>(t);
   }
-  g_dev[dev] = d;
+  g_dev[ctx] = d;
   *out = d;
   return d.ok ? SHARQ_OK : SHARQ_ERR_ARCH;
+}
+
+// Slot of `stream`: the NULL (legacy default) stream has slot 0; other streams get slots
+// 1 .. kStatusSlots-1 in the order they are first seen, round robin beyond that.
+int stream_slot(const DeviceInfo& d, cudaStream_t stream) {
+  if (stream == nullptr) return 0;
+  std::lock_guard<std::mutex> lk(g_mu);
+  const StreamKey key{d.ctx_id, stream};
+  auto it = g_stream_slot.find(key);
+  if (it != g_stream_slot.end()) return it->second;
+  int& next = g_next_slot[d.ctx_id];
+  const int slot = 1 + next % (kStatusSlots - 1);
+  ++next;
+  if (g_stream_slot.size() > 4096) g_stream_slot.clear();
+  g_stream_slot[key] = slot;
+  return slot;
+}
+
+unsigned int* status_word(const DeviceInfo& d, cudaStream_t stream) {
+  return d.status_words + stream_slot(d, stream);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -282,7 +360,7 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
   p.M = a->M;
   p.K = a->K;
   p.Mp = int(round_up(size_t(a->M), 128));
-  p.status = d.status;
+  p.status = status_word(d, st);
   p.timeout_ns = kWaitLimitNs;
   p.gamma = gamma;
   p.rstd = rstd;
@@ -327,6 +405,22 @@ __global__ void wait_probe_kernel(const uint32_t* flag, uint32_t expected, uint6
     }
     __nanosleep(1000);
   }
+}
+
+// Reads and clears status words atomically: slot >= 0 moves that slot's word into
+// taken[slot]; slot < 0 clears every slot and leaves the first non-zero word (in slot
+// order) in taken[kStatusSlots]. One thread: at most kStatusSlots atomics.
+__global__ void status_take_kernel(unsigned int* words, unsigned int* taken, int slot) {
+  if (slot >= 0) {
+    taken[slot] = atomicExch(words + slot, 0u);
+    return;
+  }
+  unsigned int first = 0;
+  for (int i = 0; i < kStatusSlots; ++i) {
+    const unsigned int v = atomicExch(words + i, 0u);
+    if (first == 0) first = v;
+  }
+  taken[kStatusSlots] = first;
 }
 }  // namespace
 }  // namespace sharq
@@ -461,11 +555,11 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   p.N = N;
   p.K = K;
   p.Mp = int(round_up(size_t(M), 128));
-  p.status = d.status;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  p.status = status_word(d, st);
   p.timeout_ns = kWaitLimitNs;
   p.splits = 1;
   p.ws = nullptr;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   const bool own = a->cfg.residual == 3;  // residual with its own tensor scale
   if (M >= 256 && N % 256 == 0 && !own) {
@@ -545,9 +639,26 @@ sharq_status sharq_wait_probe(const uint32_t* flag, uint32_t expected, uint64_t 
   DeviceInfo d;
   sharq_status s = device_info(&d);
   if (s != SHARQ_OK) return s;
-  wait_probe_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(flag, expected, limit_ns,
-                                                                   d.status);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  wait_probe_kernel<<<1, 1, 0, st>>>(flag, expected, limit_ns, status_word(d, st));
   return from_cuda(cudaGetLastError());
+}
+
+sharq_status sharq_read_device_status(void* stream) {
+  DeviceInfo d;
+  sharq_status s = device_info(&d);
+  if (s != SHARQ_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int slot = stream_slot(d, st);
+  // in stream order: after every kernel this stream launched before the call
+  status_take_kernel<<<1, 1, 0, st>>>(d.status_words, d.status_taken, slot);
+  if (cudaGetLastError() != cudaSuccess) return SHARQ_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyAsync(&v, d.status_taken + slot, sizeof(v), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return SHARQ_ERR_CUDA;
+  return v == 0 ? SHARQ_OK : static_cast<sharq_status>(v);
 }
 
 sharq_status sharq_device_status(void) {
@@ -555,11 +666,11 @@ sharq_status sharq_device_status(void) {
   sharq_status s = device_info(&d);
   if (s != SHARQ_OK) return s;
   if (cudaDeviceSynchronize() != cudaSuccess) return SHARQ_ERR_CUDA;
+  status_take_kernel<<<1, 1>>>(d.status_words, d.status_taken, -1);
+  if (cudaGetLastError() != cudaSuccess) return SHARQ_ERR_CUDA;
   unsigned int v = 0;
-  if (cudaMemcpy(&v, d.status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return SHARQ_ERR_CUDA;
-  const unsigned int zero = 0;
-  if (cudaMemcpy(d.status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+  if (cudaMemcpy(&v, d.status_taken + kStatusSlots, sizeof(v), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
     return SHARQ_ERR_CUDA;
   return v == 0 ? SHARQ_OK : static_cast<sharq_status>(v);
 }

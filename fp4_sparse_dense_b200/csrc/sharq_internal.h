@@ -86,6 +86,10 @@ struct GemmPairMaps {
 cudaError_t launch_gemm_pair(const GemmPairMaps& maps, const GemmParams& p, int fmt, int mask,
                              bool residual, bool out_f32, int num_sms, cudaStream_t st);
 
+// Unique id of the current CUDA context (initialises the primary context if none is
+// current); per-context caches key on it.
+sharq_status current_context_id(unsigned long long* id);
+
 // masks whose backbone is stored compressed and runs through the sparse MMA
 inline bool is_pair_mask(int mask) {
   return mask == SHARQ_MASK_PAIR_4_8 || mask == SHARQ_MASK_PAIR_4_8_GIVEN;

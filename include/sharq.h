@@ -15,13 +15,14 @@
  *   never allocates or frees device memory and keeps no pointer after a call returns,
  *   except a small host-side cache of TMA descriptors keyed by (pointer, shape).
  * - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy default
- *   stream) and the call returns without synchronising, except sharq_device_status().
+ *   stream) and the call returns without synchronising, except the two status reads.
  * - Every device pointer must be 16-byte aligned (TMA / 128-bit access); a misaligned
  *   pointer returns SHARQ_ERR_MISALIGNED before anything is enqueued.
  * - Shapes: K % 256 == 0, N % 128 == 0, M >= 1 (no upper bound other than int32 sizes).
  * - Errors are returned by value; no call aborts the process. A CUDA launch error is
  *   reported as SHARQ_ERR_CUDA. A kernel that gives up on a bounded wait records
- *   SHARQ_ERR_TIMEOUT in a device status word read back by sharq_device_status().
+ *   SHARQ_ERR_TIMEOUT in the status word of its stream, read back by
+ *   sharq_read_device_status(stream) (or, device-wide, sharq_device_status()).
  * - The library needs an sm_100 device (B200); on anything else the compute calls return
  *   SHARQ_ERR_ARCH. The size queries and sharq_status_string need no GPU.
  */
@@ -243,7 +244,9 @@ SHARQ_API sharq_status sharq_linear_workspace_size(int32_t M, int32_t N, int32_t
  * - A shape whose split-K scratch would exceed 16 MiB returns SHARQ_ERR_UNSUPPORTED
  *   (use sharq_linear with a workspace of sharq_linear_workspace_size bytes instead).
  * - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *   with that device current); make that first call before any stream capture.
+ *   with that device current) and caches it per CUDA context, so a device reset (a new
+ *   context) triggers a fresh lookup; make the first call in each context before any stream
+ *   capture.
  * - Every call uses the same array and leaves its partial sums there; nothing in it has to
  *   start at zero (each call overwrites every value it reads). Calls that overlap on the
  *   GPU (different streams, or different host threads) race on the array. */
@@ -252,16 +255,28 @@ SHARQ_API sharq_status sharq_linear_noalloc(const sharq_act* act, const sharq_we
 
 /* Failure-detection self-test (no counterpart in the pages): launches one thread that
  * waits until the device word *flag equals `expected`, for at most limit_ns nanoseconds
- * (1 ms ... 10 s). On expiry it records SHARQ_ERR_TIMEOUT in the device status word and
- * returns, exactly as the GEMM's bounded pipeline waits do, so that a test can exercise
- * the detection path (sharq_device_status reports the timeout, the context stays usable)
- * without a fault. flag: device pointer, 4-byte aligned. Asynchronous on `stream`. */
+ * (1 ms ... 10 s). On expiry it records SHARQ_ERR_TIMEOUT in the status word of `stream`
+ * and returns, exactly as the GEMM's bounded pipeline waits do, so that a test can exercise
+ * the detection path (sharq_read_device_status reports the timeout, the context stays
+ * usable) without a fault. flag: device pointer, 4-byte aligned. Asynchronous on `stream`. */
 SHARQ_API sharq_status sharq_wait_probe(const uint32_t* flag, uint32_t expected,
                                         uint64_t limit_ns, void* stream);
 
-/* Synchronises the device, returns and clears the status word the kernels write on a
- * bounded-wait timeout (SHARQ_OK or SHARQ_ERR_TIMEOUT), or SHARQ_ERR_CUDA if the
- * synchronisation itself fails. */
+/* Status of the work enqueued on `stream` (no counterpart in the pages: failure detection).
+ * A kernel that gives up on a bounded wait records SHARQ_ERR_TIMEOUT in the status word of
+ * the stream it was launched on (one word per stream: the NULL stream has its own, the
+ * first 63 other streams a context uses get one each, further streams share them round
+ * robin). This call enqueues a one-thread kernel on `stream` that reads and clears that word
+ * in one atomic exchange, copies the value back on `stream` and synchronises `stream` only
+ * (other streams keep running). Returns SHARQ_OK or SHARQ_ERR_TIMEOUT for the work enqueued
+ * on `stream` before the call (each timeout is reported once), or SHARQ_ERR_CUDA if the
+ * launch, copy or synchronisation fails. Work on another stream that shares the slot
+ * reports to it as well. Not for use while `stream` is being captured into a graph. */
+SHARQ_API sharq_status sharq_read_device_status(void* stream);
+
+/* Device-wide variant: synchronises the device, then reads and clears every stream's status
+ * word (atomically, one exchange per word) and returns the first non-zero one (SHARQ_OK if
+ * none), or SHARQ_ERR_CUDA if the synchronisation fails. */
 SHARQ_API sharq_status sharq_device_status(void);
 
 /* Static, human-readable name of a status code. */

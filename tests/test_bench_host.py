@@ -47,3 +47,48 @@ def test_input_sets_exceed_l2(bench):
         assert n >= 3 and n * (M * K + M * N) * 2 >= 2.5 * bench.L2_BYTES
     assert bench.input_sets(4096, 4096, 14336) == 3  # the default workload is unchanged
     assert bench.input_sets(1, 14336, 4096) == 3     # decode rotates its weights instead
+
+
+def test_stack_layout_covers_the_seven_linears(bench):
+    fused, fgroups = bench.stack_layout(False)
+    unfused, ugroups = bench.stack_layout(True)
+    flops = lambda sh: sum(k * n for k, n in sh.values())  # noqa: E731
+    assert flops(fused) == flops(unfused)  # concatenation along N keeps the work
+    assert set(fused) == {"qkv", "o", "gate_up", "down"} and len(unfused) == 7
+    for shapes, groups in ((fused, fgroups), (unfused, ugroups)):
+        names = [nm for _, _, nms in groups for nm in nms]
+        assert sorted(names) == sorted(shapes)
+        for _, K, nms in groups:
+            assert all(shapes[nm][0] == K for nm in nms)
+
+
+def test_stack_cpu_sample_counts_what_it_ran(bench):
+    """The reference arm's layer sample: whole passes over every linear, FLOPs counted from
+    the rows and columns actually multiplied."""
+    args = argparse.Namespace(unfused=False, fmt="nvfp4", mask="pair48", residual="on")
+    samples = bench.reference_stack_samples(args, 11)
+    assert [s["name"] for s in samples] == ["qkv", "o", "gate_up", "down"]
+    for s in samples:
+        assert s["x"].shape == (bench.STACK_CPU_ROWS, s["K"])
+        assert s["qw"].wq.shape == (bench.STACK_CPU_COLS, s["K"])
+    v, passes, t, rows = bench.time_stack_passes(samples, 0.0, bench.oracle_modes(args))
+    assert passes == 1 and rows == bench.STACK_CPU_ROWS and v > 0
+    flops = sum(2.0 * rows * bench.STACK_CPU_COLS * s["K"] for s in samples)
+    assert abs(v - flops / t / 1e12) < 1e-9
+
+
+def test_reference_arm_reports_the_time_it_ran(bench, capsys, monkeypatch):
+    """ms_per_step is the real duration of a sample step, so steps x ms_per_step is the
+    CPU time the arm spent (not an extrapolation to a full-size step)."""
+    import json
+    import time
+    monkeypatch.setenv("RANK", "0")
+    args = argparse.Namespace(workload="stack8b", m=None, unfused=False, fmt="nvfp4",
+                              mask="pair48", residual="on", steps=2, warmup=1, gpus=1)
+    t0 = time.perf_counter()
+    assert bench.run_reference(args) == 0
+    wall = time.perf_counter() - t0
+    d = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["steps"] == 2
+    assert d["steps"] * d["ms_per_step"] * 1e-3 <= wall
+    assert d["config"]["workload"] == "stack8b" and d["config"]["M"] == 8192

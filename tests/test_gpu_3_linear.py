@@ -152,7 +152,8 @@ def test_full_size_sampled_outputs(name, M, K, N, per_row):
     check_y(y[np.ix_(rows, cols)], y64, True)
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 14336, 4096), (8, 14336, 4096), (16, 4096, 1024),
+@pytest.mark.parametrize("M,K,N", [(1, 14336, 4096), (8, 14336, 4096), (16, 14336, 4096),
+                                   (16, 4096, 1024),
                                    (64, 14336, 4096), (100, 2048, 384)])
 def test_split_k_decode(M, K, N):
     """Decode-sized M: the split-K path (caller workspace, fixed-order reduction) agrees with

@@ -37,7 +37,8 @@ def _rel(a, b):
     return float((a - b).norm() / b.norm())
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 14336, 4096), (64, 14336, 4096), (8, 4096, 1024)])
+@pytest.mark.parametrize("M,K,N", [(1, 14336, 4096), (16, 14336, 4096), (64, 14336, 4096),
+                                   (8, 4096, 1024)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_noalloc_matches_linear_on_two_calls(M, K, N, out):
     sq, torch, act, wt = _setup(M, K, N)
