@@ -845,17 +845,18 @@ def run_stack(args):
     stream = torch.cuda.current_stream()
 
     def layer(i, ev=None):
+        """ev: ({group: (start, end)} around the preparations, {linear: end} after the GEMMs)."""
         lw = QW[i % layers]
         for gname, _, names in groups:
             if ev is not None:
-                ev[gname][0].record(stream)
+                ev[0][gname][0].record(stream)
             a = sq.prepare(X[gname], cfg, out=A[gname])
             if ev is not None:
-                ev[gname][1].record(stream)
+                ev[0][gname][1].record(stream)
             for nm in names:
                 sq.linear(a, lw[nm], out=Y[nm], workspace=WS[nm])
                 if ev is not None:
-                    ev[nm].record(stream)
+                    ev[1][nm].record(stream)
 
     ng = len(groups)
 
@@ -918,20 +919,20 @@ def run_stack(args):
     n_ev = max(1, min(args.steps, 50))
     evs = []
     for i in range(n_ev):
-        ev = {gname: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for gname, _, _ in groups}
-        ev.update({nm: torch.cuda.Event(enable_timing=True) for nm in shapes})
+        ev = ({gname: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for gname, _, _ in groups},
+              {nm: torch.cuda.Event(enable_timing=True) for nm in shapes})
         layer(i, ev)
         evs.append(ev)
     torch.cuda.synchronize()
-    prep_ms = {gname: float(np.mean([e[gname][0].elapsed_time(e[gname][1]) for e in evs]))
+    prep_ms = {gname: float(np.mean([e[0][gname][0].elapsed_time(e[0][gname][1]) for e in evs]))
                for gname, _, _ in groups}
     gemm_ms = {}
     for gname, _, names in groups:
-        prev = [e[gname][1] for e in evs]
+        prev = [e[0][gname][1] for e in evs]
         for nm in names:
-            gemm_ms[nm] = float(np.mean([p.elapsed_time(e[nm]) for p, e in zip(prev, evs)]))
-            prev = [e[nm] for e in evs]
+            gemm_ms[nm] = float(np.mean([p.elapsed_time(e[1][nm]) for p, e in zip(prev, evs)]))
+            prev = [e[1][nm] for e in evs]
 
     # each preparation alone, calls back to back over copies of its input larger than L2
     # together (X read from HBM every call)
