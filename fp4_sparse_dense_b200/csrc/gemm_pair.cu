@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       uint32_t ph = 0;
       bool ok = true;
       for (int t = cluster; t < pair_tiles && ok; t += n_clusters) {
-        const int mb2 = t % tiles_m2, nb = t / tiles_m2;
+        const int mb2 = p.n_fast ? t / p.tiles_n : t % tiles_m2;
+        const int nb = p.n_fast ? t % p.tiles_n : t / tiles_m2;
         const int rb = mb2 * 2 + int(rank);               // this CTA's 128-row block
         const int rb_sf = rb < last_rb ? rb : last_rb;    // in-bounds block for scales
         for (int kt = 0; kt < KT; ++kt) {
@@ -302,7 +303,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     int tcount = 0;
     bool ok = true;
     for (int t = cluster; t < pair_tiles; t += n_clusters, ++tcount) {
-      const int mb2 = t % tiles_m2, nb = t / tiles_m2;
+      const int mb2 = p.n_fast ? t / p.tiles_n : t % tiles_m2;
+      const int nb = p.n_fast ? t % p.tiles_n : t / tiles_m2;
       if (!ptx::mbar_wait(ptx::smem_u32(tfull_bar), uint32_t(tcount) & 1u, abort_flag, limit)) {
         ok = false;
         break;

@@ -559,6 +559,7 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   p.status = status_word(d, st);
   p.timeout_ns = kWaitLimitNs;
   p.splits = 1;
+  p.n_fast = 0;
   p.ws = nullptr;
 
   const bool own = a->cfg.residual == 3;  // residual with its own tensor scale
@@ -596,6 +597,16 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
     if (pair && !res) pm.wsd = pm.wss;
     p.tiles_m = (M + 127) / 128;
     p.tiles_n = N / 256;
+    // Raster order: the operand whose whole payload is smaller stays in L2 while the other
+    // streams through once. With M fastest every wave touches all activation rows (reused
+    // across the weight's column tiles), with N fastest every wave touches the whole weight.
+    {
+      const double act_bytes = double(asz.bq) + double(asz.bs) + double(asz.bm) +
+                               double(asz.rq) + double(asz.rs);
+      const double w_bytes = double(wsz.codes) + double(wsz.scales_dense) +
+                             double(pair ? wsz.scales_sparse : 0);
+      p.n_fast = act_bytes > w_bytes ? 1 : 0;
+    }
     return from_cuda(launch_gemm_pair(pm, p, a->cfg.fmt, a->cfg.mask, res, y_dtype == SHARQ_F32,
                                       d.num_sms, st));
   }

@@ -54,6 +54,10 @@ struct GemmParams {
   void* Y;
   int M, N, K, Mp;
   int tiles_m, tiles_n;
+  // tile order of the persistent CTA-pair kernel: 0 = M fastest (consecutive tiles share a
+  // weight tile; the whole activation operand is reused from L2 across the N columns),
+  // 1 = N fastest (consecutive tiles share activation rows; the whole weight is reused)
+  int n_fast;
   int splits;  // K ranges per output tile (1: no split; >1: partials in ws, then a reduction)
   float* ws;   // split-K partials [splits][M][N] (caller-owned workspace)
   unsigned int* status;
