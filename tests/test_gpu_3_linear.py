@@ -59,6 +59,12 @@ PAIR_CASES = [  # M >= 256 and N % 256 == 0: the CTA-pair kernel (odd 128-row co
     ("nvfp4", "elem24", True, 384, 512, 256),
     ("mxfp4", "pair48", True, 513, 512, 256),
     ("mxfp4", "elem24", True, 256, 256, 512),
+    # 80 pair tiles for 74 CTA pairs: some pairs run a second tile (K / 256 even, so the
+    # next tile's scales are copied while the epilogue drains the accumulator)
+    ("nvfp4", "pair48", True, 2048, 512, 2560),
+    ("nvfp4", "pair48", False, 2048, 512, 2560),
+    ("mxfp4", "pair48", True, 2048, 512, 2560),
+    ("nvfp4", "elem24", True, 2048, 512, 2560),
 ]
 MX_CASES = [
     ("mxfp4", "pair48", True, 128, 512, 256),
