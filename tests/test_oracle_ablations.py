@@ -128,3 +128,19 @@ def test_two_accumulator_product_is_sparse_part_plus_plain_nvfp4_of_the_residual
     sparse = S.linear_sparse_only(p, qw)
     plain_r = S.linear(S.prepare(p.r, S.NVFP4, S.NONE, residual=False), qw)
     np.testing.assert_allclose(y, sparse + plain_r, rtol=1e-12, atol=1e-12 * np.abs(y).max())
+
+
+def test_weight_block_study_orders_the_errors():
+    """The 32-element weight block that lets one FP4 payload serve both scale views costs
+    weight accuracy against 16-element NVFP4 blocks: its weight error is larger (each scale
+    covers twice the values), and the Y error follows; both sit above the activations'
+    own share (activations quantised, weight exact)."""
+    from oracle import weight_block_study as WB
+    from workloads import gaussian_weight
+    rng = np.random.default_rng(5)
+    x = heavy_activations(rng, 32, 1024).values
+    w = gaussian_weight(rng, 1024, 512).values
+    r = WB.study(x, w)
+    assert r["16"]["w_err"] < r["32"]["w_err"] < 0.2
+    assert r["16"]["y_err"] < r["32"]["y_err"]
+    assert r["act_only_y_err"] < r["16"]["y_err"]
