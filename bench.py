@@ -555,11 +555,36 @@ def run_gpu(args, emit: bool = True, light: bool = False):
     if args.pipeline:  # warm the two-stream schedule too
         timed_steps(args.warmup)
         torch.cuda.synchronize()
+    # Decode-sized steps (a few microseconds each) outrun the host's launches: they are
+    # replayed from CUDA graphs (the same kernels with the same programmatic dependencies,
+    # no host calls in the timed region), so the numbers are device time.
+    use_graph = decode and not args.pipeline
+
+    def captured(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    g_steps = captured(lambda: timed_steps(args.steps)) if use_graph else None
     with Clocks(local) as clk:
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         t_start.record(stream)
-        timed_steps(args.steps)
+        if g_steps is not None:
+            g_steps.replay()
+        else:
+            timed_steps(args.steps)
         t_end.record(stream)
         torch.cuda.synchronize()
     if world > 1:
@@ -568,18 +593,29 @@ def run_gpu(args, emit: bool = True, light: bool = False):
     ms_max = max_over_ranks(ms, dist, dev)
 
     # per-kernel durations for the roofline: a second pass with events around each call on
-    # the launching stream
+    # the launching stream; for graph-replayed decode steps, a graph of the preparations
+    # alone, the linear call's time being the rest of the step
     n_ev = min(args.steps, 200)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
-    for i in range(n_ev):
-        ev[i][0].record(stream)
-        a = step(i)
-        ev[i][1].record(stream)
-        sq.linear(a, QW[i % n_w], out=Y[i % n_sets], workspace=WS)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    prep_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    if use_graph:
+        del g_steps
+        g_prep = captured(lambda: [step(i) for i in range(n_ev)])
+        g_step = captured(lambda: timed_steps(n_ev))
+        t_prep = timed(g_prep.replay) / n_ev
+        t_step = timed(g_step.replay) / n_ev
+        del g_prep, g_step
+        prep_ms = [t_prep] * n_ev
+        gemm_ms = [t_step - t_prep] * n_ev
+    else:
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
+        for i in range(n_ev):
+            ev[i][0].record(stream)
+            a = step(i)
+            ev[i][1].record(stream)
+            sq.linear(a, QW[i % n_w], out=Y[i % n_sets], workspace=WS)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        prep_ms = [e[0].elapsed_time(e[1]) for e in ev]
+        gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
 
     # the preparation alone, calls back to back (as in a layer, where each one's launch hides
     # behind the previous kernel) over enough input sets that every call reads X from HBM
@@ -598,13 +634,15 @@ def run_gpu(args, emit: bool = True, light: bool = False):
     for j in range(n_prep):
         sq.prepare(XP[j], cfg, out=AP[j], amax=AMP[j])
     torch.cuda.synchronize()
-    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    p0.record(stream)
-    for j in range(n_pc):
-        sq.prepare(XP[j % n_prep], cfg, out=AP[j % n_prep], amax=AMP[j % n_prep])
-    p1.record(stream)
-    torch.cuda.synchronize()
-    prep_b2b = p0.elapsed_time(p1) / n_pc
+    def prep_calls():
+        for j in range(n_pc):
+            sq.prepare(XP[j % n_prep], cfg, out=AP[j % n_prep], amax=AMP[j % n_prep])
+    if use_graph:
+        g_pc = captured(prep_calls)
+        prep_b2b = timed(g_pc.replay) / n_pc
+        del g_pc
+    else:
+        prep_b2b = timed(prep_calls) / n_pc
     del XP, AP
     flops = 2.0 * M * N * K
     value = job_throughput(flops, world, args.steps, ms_max)
@@ -736,6 +774,8 @@ def single_line(args, world, M, K, N, n_sets, n_w, wbytes, decode, WS, flops, va
                               " MB of X and Y > 126 MB L2)"),
                        "schedule": ("pipelined: step i+1's preparation beside step i's GEMM "
                                     "(two streams)") if args.pipeline else "serial",
+                       "launch": ("steps replayed from a CUDA graph (decode-sized calls outrun "
+                                  "host launches)") if decode and not args.pipeline else "eager",
                        "amax": "given (reduced before the timed region)" if args.given_amax
                                else "reduced in every call",
                        "parallelism": f"dp{world}"},
@@ -880,7 +920,7 @@ def run_stack(args):
     torch.cuda.synchronize()
     assert sq.sharq_device_status() == 0
     graph = None
-    if args.graph:
+    if args.graph or M < 256:  # decode-sized layers outrun host launches: replay a graph
         # one CUDA graph of `layers` layers (every weight set once): replaying it launches
         # the same kernels with the same programmatic dependencies, without the host calls
         if args.steps % layers:
@@ -1006,7 +1046,8 @@ def run_stack(args):
                     "x U[20,50] redrawn per row; W ~ N(0, 0.02), random init)",
             "config": {"workload": "stack8b", "M": M, "fused": not args.unfused,
                        "schedule": "pipelined" if args.pipeline else "serial",
-                       "launch": f"CUDA graph of {layers} layers" if args.graph else "eager",
+                       "launch": (f"CUDA graph of {layers} layers" if args.graph or M < 256
+                                  else "eager"),
                        "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
                        "layers_rotated": layers, "format": args.fmt, "mask": args.mask,
                        "residual": args.residual, "out": "bf16",

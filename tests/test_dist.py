@@ -54,3 +54,36 @@ def test_single_process_reduction_is_identity():
     import bench
     assert bench.max_over_ranks(5.0, None, "cpu") == 5.0
     assert bench.job_throughput(1e12, 1, 1, 1000.0) == pytest.approx(1.0)
+
+
+def _ref_worker(rank, world, q):
+    import argparse
+    import contextlib
+    import io
+    sys.path.insert(0, ROOT)
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world))
+    import bench
+    args = argparse.Namespace(workload="stack8b", m=None, unfused=False, fmt="nvfp4",
+                              mask="pair48", residual="on", steps=1, warmup=1, gpus=world)
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        rc = bench.run_reference(args)
+    q.put((rank, rc, out.getvalue()))
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under torchrun the reference arm (the CPU oracle) runs and prints on rank 0 only; the
+    other ranks exit 0 without work or output."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_ref_worker, args=(r, 2, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(300)
+        assert p.exitcode == 0
+    res = dict((r, (rc, txt)) for r, rc, txt in (q.get(timeout=5) for _ in range(2)))
+    assert res[1] == (0, "")
+    rc0, txt0 = res[0]
+    lines = [ln for ln in txt0.splitlines() if ln.startswith("{")]
+    assert rc0 == 0 and len(lines) == 1 and '"impl": "reference"' in lines[0]

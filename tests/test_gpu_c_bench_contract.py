@@ -87,6 +87,7 @@ def test_bench_decode_rows():
     the split-K summing kernel is counted among the launches."""
     d = _run("--workload", "mlp_down", "--m", "1")
     assert d["config"]["M"] == 1 and d["config"]["workload"] == "mlp_down"
+    assert "CUDA graph" in d["config"]["launch"]  # device time, not host launch latency
     assert "copies" in d["config"]["l2"]
     r = d["roofline"]
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["split_k"] is True
