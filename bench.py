@@ -778,6 +778,7 @@ def single_line(args, world, M, K, N, n_sets, n_w, wbytes, decode, WS, flops, va
                                   "host launches)") if decode and not args.pipeline else "eager",
                        "amax": "given (reduced before the timed region)" if args.given_amax
                                else "reduced in every call",
+                       "gemm_workspace": "split-K" if WS is not None else "none",
                        "parallelism": f"dp{world}"},
             "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": peak,
                          "unit": "TFLOP/s", "frac": gemm_tflops / peak,
@@ -811,9 +812,10 @@ def single_line(args, world, M, K, N, n_sets, n_w, wbytes, decode, WS, flops, va
             "pct_fp4_peak": 100.0 * gemm_tflops / peak,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
                     "d2h_bytes_per_step": M * N * 2},
+            # split-K (decode-sized M) adds a summing kernel
             "gpu_launches": (len(prep_kernels(args.fmt, args.mask, args.residual,
                                               args.given_amax)) + 1 +
-                             (1 if WS is not None else 0)) * args.steps,
+                             (1 if WS is not None and decode else 0)) * args.steps,
             "clocks": clocks,
         }
         if decode:  # below the ridge point the GEMM streams its weight: an HBM roofline
@@ -1050,6 +1052,8 @@ def run_stack(args):
                                   else "eager"),
                        "linears": [f"{nm} {k}x{n}" for nm, (k, n) in shapes.items()],
                        "layers_rotated": layers, "format": args.fmt, "mask": args.mask,
+                       "gemm_workspace": {nm: "split-K" if WS[nm] is not None else "none"
+                                          for nm in shapes},
                        "residual": args.residual, "out": "bf16",
                        "l2": (f"weights rotate over {layers} layers ({layers * wbytes / 1e6:.0f} MB"
                               f"); X {sum(M * K * 2 for _, K, _ in groups) / 1e6:.0f} MB and Y "
@@ -1076,7 +1080,8 @@ def run_stack(args):
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": (sum(len(prep_kernels(args.fmt, args.mask, args.residual))
                                  for _ in groups)
-                             + sum(1 + (1 if WS[nm] is not None else 0) for nm in shapes))
+                             + sum(1 + (1 if WS[nm] is not None and M < 256 else 0)
+                                   for nm in shapes))
                             * args.steps,
             "clocks": clocks,
         }
