@@ -64,6 +64,8 @@ struct GemmCfg {
   static constexpr int STAGE_RAW = OFF_E + E_BYTES;
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int TX = STAGE_RAW;  // every byte of the stage arrives by copy
+  static constexpr int TX_W = W_BYTES + SWD_BYTES + SWS_BYTES;  // the weight's part of it
+  static constexpr int TX_A = TX - TX_W;                         // the activations' part
   static constexpr int EPI_BYTES = 8 * 2048;  // one 32 x 32 bf16 staging box per epilogue warp
   static constexpr int STAGES_FIT = (kMaxSmem - 2048 - EPI_BYTES) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
@@ -132,13 +134,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::prefetch_tensormap(&tm_b);
     if (RES) ptx::prefetch_tensormap(&tm_r);
   }
+  // the weight's part of K step kt of N block nb into stage buffer st (codes and scales)
+  auto load_w = [&](uint8_t* st, int kt, int nb, uint32_t fb) {
+    ptx::tma_load_2d(ptx::smem_u32(st + C::OFF_W), &tm_w, kt * 128, nb * BN, fb);
+    if (PAIR) {
+      for (int rb = 0; rb < BN / 128; ++rb) {
+        const uint8_t* w =
+            p.wss + (size_t(nb * (BN / 128) + rb) * (p.K / 32 / 4) + size_t(kt) * 2) * 512;
+        ptx::bulk_load(ptx::smem_u32(st + C::OFF_SWS + rb * 1024), w, 1024, fb);
+      }
+    }
+    if (C::DENSE_W) {
+      for (int rb = 0; rb < BN / 128; ++rb) {
+        const uint8_t* w = p.wsd + (size_t(nb * (BN / 128) + rb) * (p.K / C::GD / 4) +
+                                    size_t(kt) * C::DCH) * 512;
+        ptx::bulk_load(ptx::smem_u32(st + C::OFF_SWD + rb * C::DCH * 512), w, C::DCH * 512, fb);
+      }
+    }
+  };
+  // Decode-sized M: the weight part of the first tile's first stages is loaded now, while the
+  // kernel launched just before (the preparation) may still run. The weight is not among its
+  // outputs: it was written before that kernel started (sharq_linear's contract). The
+  // stages' barriers only get the bytes to expect here; their arrival, with the
+  // activations' bytes, comes after the wait, so no stage completes early.
+  int n_pre = 0;
+  if (p.prefetch_w && warp == 0) {
+    if (lane == 0 && int(blockIdx.x) < tiles) {
+      const int t = blockIdx.x;
+      const int tmn = t % tiles_mn, ks = t / tiles_mn;
+      const int nb = tmn / p.tiles_m;
+      const int kt0 = ks * KT / p.splits, kt1 = (ks + 1) * KT / p.splits;
+      n_pre = kt1 - kt0 < C::STAGES ? kt1 - kt0 : C::STAGES;
+      for (int i = 0; i < n_pre; ++i) {
+        const uint32_t fb = ptx::smem_u32(full_bar + i);
+        ptx::mbar_expect_tx(fb, C::TX_W);
+        load_w(smem + i * C::STAGE, kt0 + i, nb, fb);
+      }
+    }
+    n_pre = __shfl_sync(0xFFFFFFFFu, n_pre, 0);
+  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint64_t limit = p.timeout_ns;
   // launched as a programmatic dependent: the set-up above overlapped the previous kernel;
-  // nothing it wrote (the operands) is read before this point
+  // nothing it wrote (the activation operands) is read before this point
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
 
@@ -148,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      bool first = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, first = false) {
         const int tmn = t % tiles_mn, ks = t / tiles_mn;
         const int mb = tmn % p.tiles_m, nb = tmn / p.tiles_m;
         const int kt0 = ks * KT / p.splits, kt1 = (ks + 1) * KT / p.splits;
@@ -158,9 +200,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t fb = ptx::smem_u32(full_bar + s);
-          ptx::mbar_arrive_expect_tx(fb, C::TX);
           uint8_t* st = smem + s * C::STAGE;
-          ptx::tma_load_2d(ptx::smem_u32(st + C::OFF_W), &tm_w, kt * 128, nb * BN, fb);
+          if (first && kt - kt0 < n_pre) {  // weight part already on its way (see above)
+            ptx::mbar_arrive_expect_tx(fb, C::TX_A);
+          } else {
+            ptx::mbar_arrive_expect_tx(fb, C::TX);
+            load_w(st, kt, nb, fb);
+          }
           if (RES) ptx::tma_load_2d(ptx::smem_u32(st + C::OFF_R), &tm_r, kt * 128, mb * 128, fb);
           ptx::tma_load_2d(ptx::smem_u32(st + C::OFF_B), &tm_b, kt * (PAIR ? 64 : 128), mb * 128,
                            fb);
@@ -173,22 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::bulk_load(ptx::smem_u32(st + C::OFF_SFB), src, C::SFB_BYTES, fb);
             const uint8_t* e = p.bm + size_t(kt) * p.Mp * 16 + size_t(mb) * 2048;
             ptx::bulk_load(ptx::smem_u32(st + C::OFF_E), e, 2048, fb);
-            for (int rb = 0; rb < BN / 128; ++rb) {
-              const uint8_t* w =
-                  p.wss + (size_t(nb * (BN / 128) + rb) * (p.K / 32 / 4) + size_t(kt) * 2) * 512;
-              ptx::bulk_load(ptx::smem_u32(st + C::OFF_SWS + rb * 1024), w, 1024, fb);
-            }
           } else {
             const uint8_t* src = p.bs + (size_t(mb) * (p.K / C::GD / 4) + size_t(kt) * C::DCH) * 512;
             ptx::bulk_load(ptx::smem_u32(st + C::OFF_SFB), src, C::SFB_BYTES, fb);
-          }
-          if (C::DENSE_W) {
-            for (int rb = 0; rb < BN / 128; ++rb) {
-              const uint8_t* w = p.wsd + (size_t(nb * (BN / 128) + rb) * (p.K / C::GD / 4) +
-                                          size_t(kt) * C::DCH) * 512;
-              ptx::bulk_load(ptx::smem_u32(st + C::OFF_SWD + rb * C::DCH * 512), w, C::DCH * 512,
-                             fb);
-            }
           }
           if (++s == C::STAGES) { s = 0; ph ^= 1u; }
         }

@@ -78,7 +78,16 @@ struct StreamKeyHash {
     return size_t(k.ctx * 0x9E3779B97F4A7C15ull) ^ reinterpret_cast<size_t>(k.stream);
   }
 };
-std::unordered_map<StreamKey, int, StreamKeyHash> g_stream_slot;
+// Per stream: its status slot, and whether the GEMM may load its weight before waiting for
+// the kernel launched just before it. That holds when the last launch of this library on the
+// stream was a preparation or a linear call: each of their kernels waits for its own
+// predecessor before it lets a dependent start, and none of them writes a weight. It does not
+// hold on a stream not seen before, nor after sharq_quantize_weight.
+struct StreamState {
+  int slot = 0;
+  bool weight_early = false;
+};
+std::unordered_map<StreamKey, StreamState, StreamKeyHash> g_streams;
 std::unordered_map<unsigned long long, int> g_next_slot;  // context id -> next slot to hand out
 
 sharq_status device_info(DeviceInfo* out) {
@@ -114,20 +123,35 @@ sharq_status device_info(DeviceInfo* out) {
   return d.ok ? SHARQ_OK : SHARQ_ERR_ARCH;
 }
 
-// Slot of `stream`: the NULL (legacy default) stream has slot 0; other streams get slots
-// 1 .. kStatusSlots-1 in the order they are first seen, round robin beyond that.
-int stream_slot(const DeviceInfo& d, cudaStream_t stream) {
-  if (stream == nullptr) return 0;
-  std::lock_guard<std::mutex> lk(g_mu);
+// State of `stream` (g_mu held). The NULL (legacy default) stream has slot 0; other streams
+// get slots 1 .. kStatusSlots-1 in the order they are first seen, round robin beyond that.
+StreamState& stream_state_locked(const DeviceInfo& d, cudaStream_t stream) {
   const StreamKey key{d.ctx_id, stream};
-  auto it = g_stream_slot.find(key);
-  if (it != g_stream_slot.end()) return it->second;
-  int& next = g_next_slot[d.ctx_id];
-  const int slot = 1 + next % (kStatusSlots - 1);
-  ++next;
-  if (g_stream_slot.size() > 4096) g_stream_slot.clear();
-  g_stream_slot[key] = slot;
-  return slot;
+  auto it = g_streams.find(key);
+  if (it != g_streams.end()) return it->second;
+  if (g_streams.size() > 4096) g_streams.clear();
+  StreamState st;
+  if (stream != nullptr) {
+    int& next = g_next_slot[d.ctx_id];
+    st.slot = 1 + next % (kStatusSlots - 1);
+    ++next;
+  }
+  return g_streams.emplace(key, st).first->second;
+}
+
+int stream_slot(const DeviceInfo& d, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return stream_state_locked(d, stream).slot;
+}
+
+// Records the kind of this library's latest launch on `stream` and returns whether the one
+// before it allowed the weight to be loaded early (see StreamState).
+bool note_launch(const DeviceInfo& d, cudaStream_t stream, bool weight_early_after) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  StreamState& st = stream_state_locked(d, stream);
+  const bool before = st.weight_early;
+  st.weight_early = weight_early_after;
+  return before;
 }
 
 unsigned int* status_word(const DeviceInfo& d, cudaStream_t stream) {
@@ -371,16 +395,21 @@ sharq_status prepare_impl(const void* X, sharq_dtype dtype, const sharq_act* a, 
   p.alongside = alongside ? 1 : 0;
   p.res_phase = 0;
   p.amax_in = amax_in;
-  if (a->cfg.residual != 3)
-    return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
-  // the residual's own tensor scale: amax|r| is a grid-wide reduction that follows the
-  // backbone's quantisation, so the quantisation runs twice (backbone + amax|r|, then the
-  // residual with s_r)
-  p.res_phase = 1;
-  if ((s = from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st))) != SHARQ_OK)
-    return s;
-  p.res_phase = 2;
-  return from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
+  if (a->cfg.residual != 3) {
+    s = from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
+  } else {
+    // the residual's own tensor scale: amax|r| is a grid-wide reduction that follows the
+    // backbone's quantisation, so the quantisation runs twice (backbone + amax|r|, then the
+    // residual with s_r)
+    p.res_phase = 1;
+    s = from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
+    if (s == SHARQ_OK) {
+      p.res_phase = 2;
+      s = from_cuda(launch_prep(p, bf16, a->cfg.fmt, a->cfg.mask, res, d.num_sms, st));
+    }
+  }
+  note_launch(d, st, s == SHARQ_OK);
+  return s;
 }
 }  // namespace
 }  // namespace sharq
@@ -464,6 +493,7 @@ sharq_status sharq_quantize_weight(const void* W, sharq_dtype dtype, const sharq
   DeviceInfo d;
   if ((s = device_info(&d)) != SHARQ_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  note_launch(d, st, false);  // a GEMM launched next must not read this weight early
   const bool bf16 = dtype == SHARQ_BF16;
   if (w->cfg.fmt == SHARQ_NVFP4) {
     if (cudaMemsetAsync(w->tensor_scale + 1, 0, sizeof(float), st) != cudaSuccess)
@@ -560,6 +590,7 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   p.timeout_ns = kWaitLimitNs;
   p.splits = 1;
   p.n_fast = 0;
+  p.prefetch_w = 0;
   p.ws = nullptr;
 
   const bool own = a->cfg.residual == 3;  // residual with its own tensor scale
@@ -638,6 +669,11 @@ sharq_status sharq_linear(const sharq_act* a, const sharq_weight* w, void* Y, sh
   }
   p.tiles_m = (M + 127) / 128;
   p.tiles_n = N / BN;
+  // decode-sized M: the weight stream dominates; its first stages are loaded while the
+  // kernel launched just before (normally the preparation) is still running, when that kernel
+  // is one of this library's that writes no weight (see StreamState)
+  const bool weight_early = note_launch(d, st, true);
+  p.prefetch_w = (M < 256 && weight_early) ? 1 : 0;
   if (own) return from_cuda(launch_gemm_two(maps, p, y_dtype == SHARQ_F32, d.num_sms, st));
   return from_cuda(launch_gemm(maps, p, a->cfg.fmt, a->cfg.mask, res, y_dtype == SHARQ_F32,
                                d.num_sms, st));

@@ -58,6 +58,9 @@ struct GemmParams {
   // weight tile; the whole activation operand is reused from L2 across the N columns),
   // 1 = N fastest (consecutive tiles share activation rows; the whole weight is reused)
   int n_fast;
+  // one-CTA kernel: load the weight part of the first stages before waiting for the kernel
+  // launched before it (decode-sized M, where the weight stream dominates)
+  int prefetch_w;
   int splits;  // K ranges per output tile (1: no split; >1: partials in ws, then a reduction)
   float* ws;   // split-K partials [splits][M][N] (caller-owned workspace)
   unsigned int* status;

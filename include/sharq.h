@@ -220,7 +220,15 @@ SHARQ_API sharq_status sharq_prepare_rmsnorm(const void* X, const void* gamma, f
  * the split-K path used when the output has too few tiles to occupy the GPU (decode-sized
  * M); sharq_linear_workspace_size gives the bytes it wants. With a NULL or too small
  * workspace the call runs without splitting K (same result up to summation order, slower
- * for small M). */
+ * for small M).
+ * Ordering: the GEMM is launched as a programmatic dependent of the kernel launched just
+ * before it on `stream`. It reads nothing of *act before that kernel has completed. For
+ * M < 256 it may start loading w's codes and scales while that kernel still runs, when
+ * this library's previous launch on `stream` was a preparation or a linear call. It does
+ * not do this on a stream it has not seen before, nor after sharq_quantize_weight. So w
+ * must be complete before the kernel launched just before this call starts. A caller's
+ * own kernel that writes w must not come between a preparation and this call on `stream`.
+ * A copy (cudaMemcpyAsync) or a write ordered through an event is fine. */
 SHARQ_API sharq_status sharq_linear(const sharq_act* act, const sharq_weight* w, void* Y,
                                     sharq_dtype y_dtype, void* workspace, size_t workspace_bytes,
                                     void* stream);

@@ -234,3 +234,33 @@ def test_split_k_workspace_reused_across_shapes():
         y64 = S.linear(S.prepare(x.values), qw)
         assert rel_fro(y, y64) <= 1e-5, M
 
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_weight_requantised_just_before_linear(M):
+    """At decode-sized M the GEMM may load its weight while the kernel launched just before
+    it still runs, but only when that kernel is a preparation's or a linear call's. A weight
+    re-quantised into the same buffers right before sharq_linear must be read in full: the
+    result equals that of the new weight quantised before the preparation, bit for bit, and
+    differs from the old weight's."""
+    import fp4_sparse_dense_b200 as sq
+    import torch
+    K, N = 14336, 4096
+    cfg = cfg_of("nvfp4", "pair48")
+    rng = np.random.default_rng(4242 + M)
+    x = to_device(heavy_activations(rng, M, K, per_row=True))
+    w_old = to_device(gaussian_weight(rng, K, N))
+    w_new = to_device(gaussian_weight(rng, K, N))
+    ws = sq.linear_workspace(M, N, K, cfg)
+    dt = torch.float32
+    wt = sq.quantize_weight(w_old, cfg)
+    act = sq.prepare(x, cfg)
+    y_old = sq.linear(act, wt, out_dtype=dt, workspace=ws)       # after a preparation
+    sq.quantize_weight(w_new, cfg, out=wt)                       # same buffers, new weight
+    y_late = sq.linear(act, wt, out_dtype=dt, workspace=ws)      # right after the quantisation
+    wt2 = sq.quantize_weight(w_new, cfg)
+    y_ref = sq.linear(sq.prepare(x, cfg), wt2, out_dtype=dt, workspace=ws)
+    torch.cuda.synchronize()
+    assert sq.sharq_device_status() == 0
+    assert torch.equal(y_late, y_ref)
+    assert not torch.equal(y_old, y_ref)
