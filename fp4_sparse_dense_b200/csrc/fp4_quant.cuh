@@ -193,18 +193,31 @@ __device__ __forceinline__ BlockScale nv_block_scale(float a, TensorConsts c,
   return b;
 }
 
-// decode8 for a block from nv_block_scale (sf holds the E4M3 value as an f16 pair)
+// decode8 for a block from nv_block_scale (sf holds the E4M3 value as an f16 pair):
+// (E2M1 * E4M3) * s_g per value with one float32 rounding. E2M1 * E4M3 comes from sm_100's
+// mixed-precision FMA (f16 sources; the product has at most 6 significant bits, so it is
+// exact in float32, and the -0 addend leaves it and the sign of a zero unchanged). The s_g
+// product is a packed FMA with a -0 addend: the same single rounding as a multiply. The
+// addend is formed at run time (-0 * s_g, s_g finite and >= 0) so that the compiler cannot
+// turn the FMA back into a multiply and fuse that with the caller's x - deq.
 __device__ __forceinline__ void decode8_nv(uint32_t codes, const BlockScale& b, float s_g,
                                            float* out) {
   uint32_t h[4];
   e2m1x8_to_f16x2(codes, h);
   const uint32_t sfh = __float_as_uint(b.sf);
-  const __half2 sf2 = *reinterpret_cast<const __half2*>(&sfh);
+  const float nz = __fmul_rn(-0.f, s_g);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float2 f = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[j]), sf2));
-    out[2 * j] = __fmul_rn(f.x, s_g);  // never merged into a multiply-add
-    out[2 * j + 1] = __fmul_rn(f.y, s_g);
+    float lo, hi;
+    asm("{\n\t.reg .f16 a0, a1, s0, s1;\n\t"
+        "mov.b32 {a0, a1}, %2;\n\tmov.b32 {s0, s1}, %3;\n\t"
+        "fma.rn.f32.f16 %0, a0, s0, 0f80000000;\n\t"
+        "fma.rn.f32.f16 %1, a1, s0, 0f80000000;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h[j]), "r"(sfh));
+    const float2 d = fma2_rn(make_float2(lo, hi), make_float2(s_g, s_g), make_float2(nz, nz));
+    out[2 * j] = d.x;
+    out[2 * j + 1] = d.y;
   }
 }
 
