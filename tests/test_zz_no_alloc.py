@@ -4,8 +4,8 @@ sharq_linear_noalloc is for callers that cannot allocate device memory (code cap
 CUDA graphs, allocator-free runtimes, hosts that forbid allocation on the hot path): the
 split-K scratch it needs for decode-sized M is a fixed array inside the library instead of
 a caller workspace. These tests call it through the C ABI, two calls in a row, and compare
-each result with sharq_linear given a caller-owned workspace, within the FP32 tolerance of
-the other GEMM tests. This file is collected last so that a failure here cannot hide an
+each result with sharq_linear given a caller-owned workspace, and, on two shapes, with the
+oracle's product, within the FP32 tolerance of the other GEMM tests. This file is collected last so that a failure here cannot hide an
 earlier one."""
 import ctypes
 
@@ -58,6 +58,35 @@ def test_noalloc_matches_linear_on_two_calls(M, K, N, out):
         assert not torch.isnan(y).any()
         tol = TOL_F32 if out == "f32" else 1e-3
         assert _rel(y, ref) <= tol
+
+
+@pytest.mark.parametrize("M,K,N", [(8, 4096, 1024), (16, 14336, 4096)])
+def test_noalloc_matches_oracle(M, K, N):
+    """The same calls against the oracle: its float64 product of the dequantised operands,
+    FP32 output held to the GEMM parity tests' 1e-5 relative Frobenius error."""
+    from oracle import sharq as S
+    from workloads import gaussian_weight, heavy_activations, to_device
+    import torch
+
+    import fp4_sparse_dense_b200 as sq
+    rng = np.random.default_rng(7 * M + K + N)
+    x = heavy_activations(rng, M, K, per_row=True)
+    w = gaussian_weight(rng, K, N)
+    cfg = sq.Config()
+    act = sq.prepare(to_device(x), cfg)
+    wt = sq.quantize_weight(to_device(w), cfg)
+    assert sq.linear_workspace(M, N, K, cfg) is not None  # the split-K path: library scratch
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    ca, cw = act.c(), wt.c()
+    rc = sq.sharq_linear_noalloc(ctypes.byref(ca), ctypes.byref(cw),
+                                 ctypes.c_void_p(y.data_ptr()), sq.F32,
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, sq.sharq_status_string(rc)
+    torch.cuda.synchronize()
+    assert sq.sharq_device_status() == 0
+    y64 = S.linear(S.prepare(x.values), S.quantize_weight(w.values))
+    got = y.cpu().numpy().astype(np.float64)
+    assert float(np.linalg.norm(got - y64) / np.linalg.norm(y64)) <= TOL_F32
 
 
 def test_noalloc_unsplit_shape_matches_linear():
