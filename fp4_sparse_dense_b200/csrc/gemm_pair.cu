@@ -83,6 +83,21 @@ struct PairCfg {
   static constexpr uint32_t SCALE_FMT = NV ? 0u : (1u << 23);
 };
 
+// Shared-memory matrix descriptors of one stage buffer at one add each (the MMA thread
+// issues some thirty per K step, alone in its warp, so their arithmetic is on its critical
+// path). Every address in a stage is 16-byte aligned and below 256 KB, so the descriptor's
+// 14-bit address field of base + off is the base's plus off >> 4 with no carry; the leading
+// byte offset is 16 bytes throughout. Same bits as ptx::smem_desc.
+struct StageDesc {
+  uint32_t lo;  // address field of the stage base | leading byte offset field
+  __device__ __forceinline__ explicit StageDesc(uint32_t base) : lo((base >> 4) | (1u << 16)) {}
+  template <uint32_t SBO, uint32_t LAYOUT>
+  __device__ __forceinline__ uint64_t at(uint32_t off) const {
+    constexpr uint32_t hi = ((SBO >> 4) & 0x3FFFu) | (1u << 14) | ((LAYOUT & 7u) << 29);
+    return (uint64_t(hi) << 32) | uint64_t(lo + (off >> 4));
+  }
+};
+
 }  // namespace
 
 template <int FMT, bool PAIR, bool RES, bool OUT_F32>
@@ -212,48 +227,48 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t st = ptx::smem_u32(smem + s * C::STAGE);
+          const StageDesc sd(ptx::smem_u32(smem + s * C::STAGE));
           const uint32_t tb = tbase + uint32_t(kt & 1) * C::SF_SPAN;
           // ---- scales and metadata of this K step into both CTAs' tensor memory
           if (PAIR) {
-            ptx::tmem_cp_128x128b_pair(tb + C::COL_E, ptx::smem_desc(st + C::OFF_E, 16, 128, 0));
+            ptx::tmem_cp_128x128b_pair(tb + C::COL_E, sd.at<128, 0>(C::OFF_E));
             for (int j = 0; j < 2; ++j) {
               ptx::tmem_cp_32x128b_x4_pair(tb + C::COL_SFB + 4 * j,
-                                           ptx::smem_desc(st + C::OFF_SFB + 512 * j, 16, 128, 0));
+                                           sd.at<128, 0>(C::OFF_SFB + 512 * j));
               for (int h = 0; h < 2; ++h)
                 ptx::tmem_cp_32x128b_x4_pair(
                     tb + C::COL_SWS + j * (C::BN / 32) + 4 * h,
-                    ptx::smem_desc(st + C::OFF_SWS + (h * 2 + j) * 512, 16, 128, 0));
+                    sd.at<128, 0>(C::OFF_SWS + (h * 2 + j) * 512));
             }
           } else {
             for (int c = 0; c < C::DCH; ++c)
               ptx::tmem_cp_32x128b_x4_pair(tb + C::COL_SFB + 4 * c,
-                                           ptx::smem_desc(st + C::OFF_SFB + 512 * c, 16, 128, 0));
+                                           sd.at<128, 0>(C::OFF_SFB + 512 * c));
           }
           if (RES)
             for (int c = 0; c < C::DCH; ++c)
               ptx::tmem_cp_32x128b_x4_pair(tb + C::COL_SFR + 4 * c,
-                                           ptx::smem_desc(st + C::OFF_SFR + 512 * c, 16, 128, 0));
+                                           sd.at<128, 0>(C::OFF_SFR + 512 * c));
           if (C::DENSE_W)
             for (int c = 0; c < C::DCH; ++c)
               for (int h = 0; h < 2; ++h)
                 ptx::tmem_cp_32x128b_x4_pair(
                     tb + C::COL_SWD + c * (C::BN / 32) + 4 * h,
-                    ptx::smem_desc(st + C::OFF_SWD + (h * C::DCH + c) * 512, 16, 128, 0));
+                    sd.at<128, 0>(C::OFF_SWD + (h * C::DCH + c) * 512));
           // ---- pair MMAs: backbone then residual, one accumulator
           uint32_t acc = kt > 0 ? 1u : 0u;
           if (PAIR) {
             for (int j = 0; j < 2; ++j) {
-              const uint64_t a = ptx::smem_desc(st + C::OFF_B + 32 * j, 16, 512, 4);
-              const uint64_t b = ptx::smem_desc(st + C::OFF_W + 64 * j, 16, 1024, 2);
+              const uint64_t a = sd.at<512, 4>(C::OFF_B + 32 * j);
+              const uint64_t b = sd.at<1024, 2>(C::OFF_W + 64 * j);
               ptx::mma_sp_nvf4_pair(tbase, a, b, tb + C::COL_E + 2 * j, idesc_s,
                                     tb + C::COL_SFB + 4 * j, tb + C::COL_SWS + j * (C::BN / 32), acc);
               acc = 1u;
             }
           } else {
             for (int i = 0; i < 4; ++i) {
-              const uint64_t a = ptx::smem_desc(st + C::OFF_B + 32 * i, 16, 1024, 2);
-              const uint64_t b = ptx::smem_desc(st + C::OFF_W + 32 * i, 16, 1024, 2);
+              const uint64_t a = sd.at<1024, 2>(C::OFF_B + 32 * i);
+              const uint64_t b = sd.at<1024, 2>(C::OFF_W + 32 * i);
               if (C::NV) {
                 ptx::mma_nvf4_pair(tbase, a, b, idesc_d, tb + C::COL_SFB + 4 * i,
                                    tb + C::COL_SWD + i * (C::BN / 32), acc);
@@ -268,8 +283,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           }
           if (RES) {
             for (int i = 0; i < 4; ++i) {
-              const uint64_t a = ptx::smem_desc(st + C::OFF_R + 32 * i, 16, 1024, 2);
-              const uint64_t b = ptx::smem_desc(st + C::OFF_W + 32 * i, 16, 1024, 2);
+              const uint64_t a = sd.at<1024, 2>(C::OFF_R + 32 * i);
+              const uint64_t b = sd.at<1024, 2>(C::OFF_W + 32 * i);
               if (C::NV) {
                 ptx::mma_nvf4_pair(tbase, a, b, idesc_d, tb + C::COL_SFR + 4 * i,
                                    tb + C::COL_SWD + i * (C::BN / 32), 1u);
