@@ -92,3 +92,21 @@ def test_reference_arm_reports_the_time_it_ran(bench, capsys, monkeypatch):
     assert d["impl"] == "reference" and d["steps"] == 2
     assert d["steps"] * d["ms_per_step"] * 1e-3 <= wall
     assert d["config"]["workload"] == "stack8b" and d["config"]["M"] == 8192
+
+
+def test_fp4_peak_follows_the_clock_of_the_timed_region(monkeypatch):
+    """A burst at full clock is held to 4 x the bf16 burst figure; a run under the power cap
+    (median below 90 % of the maximum clock) to 4 x the sustained figure scaled to its clock."""
+    import bench
+    monkeypatch.setattr(bench, "load_peaks", lambda: (6541.5, 1654.2, 1383.4, "measured"))
+    monkeypatch.setattr(bench, "sustained_clock_mhz", lambda: 1327.0)
+    p, src = bench.fp4_peak(1965.0, 1965.0)
+    assert p == pytest.approx(4 * 1654.2) and "burst" in src
+    p, src = bench.fp4_peak(1800.0, 1965.0)          # within 10 % of max: still a burst
+    assert p == pytest.approx(4 * 1654.2)
+    p, src = bench.fp4_peak(1515.0, 1965.0)
+    assert p == pytest.approx(4 * 1383.4 * 1515.0 / 1327.0) and "sustained" in src
+    p, src = bench.fp4_peak(None, None)              # no clock samples: the burst figure
+    assert p == pytest.approx(4 * 1654.2)
+    monkeypatch.setattr(bench, "sustained_clock_mhz", lambda: None)
+    assert bench.fp4_peak(1515.0, 1965.0)[0] == pytest.approx(4 * 1654.2)
