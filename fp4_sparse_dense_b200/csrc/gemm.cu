@@ -428,7 +428,11 @@ static cudaError_t launch_t(const GemmMaps& m, const GemmParams& p, int num_sms,
 }
 
 // Split-K reduction: Y = alpha * sum over the K ranges of the FP32 partials, in a fixed
-// order (deterministic). One thread per 8 consecutive outputs.
+// order (deterministic). One thread per 2 consecutive outputs, so that decode-sized outputs
+// spread over several SMs; the partials of up to 16 splits are loaded before any is added
+// (one L2 round trip for the usual split counts), then added in split order.
+constexpr int kReduceOut = 2;    // outputs per thread
+constexpr int kReduceBatch = 16; // splits loaded together
 template <bool OUT_F32>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ ws,
                                                             int splits, int M, int N,
@@ -436,46 +440,33 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
                                                             void* Y) {
   ptx::griddep_wait();  // the partials of the GEMM launched just before
   const size_t total = size_t(M) * N;
-  const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * kReduceOut;
   if (i >= total) return;
   const float alpha = __fmul_rn(act_ts[0], w_ts[0]);
-  // the partials of up to 8 splits are loaded together (one L2 round trip per batch, not
-  // one per split) and then added in split order, so the sum is the same fixed sequence
-  float acc[8];
-  for (int base = 0; base < splits; base += 8) {
-    float4 v[8][2];
+  float2 acc = make_float2(0.f, 0.f);
+  for (int base = 0; base < splits; base += kReduceBatch) {
+    float2 v[kReduceBatch];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (base + j < splits) {
-        const float4* src = reinterpret_cast<const float4*>(ws + size_t(base + j) * total + i);
-        v[j][0] = __ldcg(src);
-        v[j][1] = __ldcg(src + 1);
-      }
-    }
+    for (int j = 0; j < kReduceBatch; ++j)
+      if (base + j < splits)
+        v[j] = __ldcg(reinterpret_cast<const float2*>(ws + size_t(base + j) * total + i));
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kReduceBatch; ++j) {
       if (base + j >= splits) break;
-      const float t[8] = {v[j][0].x, v[j][0].y, v[j][0].z, v[j][0].w,
-                          v[j][1].x, v[j][1].y, v[j][1].z, v[j][1].w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = (base + j == 0) ? t[e] : __fadd_rn(acc[e], t[e]);
+      if (base + j == 0) {
+        acc = v[j];
+      } else {
+        acc.x = __fadd_rn(acc.x, v[j].x);
+        acc.y = __fadd_rn(acc.y, v[j].y);
+      }
     }
   }
   if (OUT_F32) {
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(Y) + i);
-    dst[0] = make_float4(__fmul_rn(acc[0], alpha), __fmul_rn(acc[1], alpha),
-                         __fmul_rn(acc[2], alpha), __fmul_rn(acc[3], alpha));
-    dst[1] = make_float4(__fmul_rn(acc[4], alpha), __fmul_rn(acc[5], alpha),
-                         __fmul_rn(acc[6], alpha), __fmul_rn(acc[7], alpha));
+    *reinterpret_cast<float2*>(static_cast<float*>(Y) + i) =
+        make_float2(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha));
   } else {
-    uint32_t w4[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(acc[2 * h], alpha),
-                                                      __fmul_rn(acc[2 * h + 1], alpha));
-      w4[h] = *reinterpret_cast<const uint32_t*>(&b2);
-    }
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(Y) + i) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha));
+    *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(Y) + i) = b2;
   }
 }
 
@@ -521,7 +512,7 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmParams& p, int fmt, int 
                          : launch_m<SHARQ_MXFP4>(maps, p, mask, residual, out_f32, num_sms, st);
   if (e != cudaSuccess || p.splits <= 1) return e;
   const size_t total = size_t(p.M) * p.N;
-  const unsigned blocks = unsigned((total / 8 + 255) / 256);
+  const unsigned blocks = unsigned((total / kReduceOut + 255) / 256);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
   cfg.blockDim = dim3(256);
