@@ -160,7 +160,10 @@ def test_full_size_sampled_outputs(name, M, K, N, per_row):
 
 @pytest.mark.parametrize("M,K,N", [(1, 14336, 4096), (8, 14336, 4096), (16, 14336, 4096),
                                    (16, 4096, 1024),
-                                   (64, 14336, 4096), (100, 2048, 384)])
+                                   (64, 14336, 4096), (100, 2048, 384),
+                                   # 16, 17 and 28 K ranges: the summing kernel loads the
+                                   # partials of up to 16 splits per batch
+                                   (2, 8192, 256), (3, 8704, 256), (1, 14336, 128)])
 def test_split_k_decode(M, K, N):
     """Decode-sized M: the split-K path (caller workspace, fixed-order reduction) agrees with
     the oracle and with the unsplit path, and repeats bit-identically."""
