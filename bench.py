@@ -753,98 +753,97 @@ def single_line(args, world, M, K, N, n_sets, n_w, wbytes, decode, WS, flops, va
     """The JSON line of a single-linear workload (rank 0)."""
     import torch
     has_res = args.residual != "off"
-    if True:
-        hbm, bf16, bf16_sus, peak_src = load_peaks()
-        clocks = clk.summary()
-        peak, peak_source = fp4_peak(clocks.get("sm_mhz"), clocks.get("sm_max_mhz"))
-        gemm_avg = float(np.mean(gemm_ms))
-        prep_avg = prep_b2b
-        prep_in_step = float(np.mean(prep_ms))
-        gemm_tflops = flops / (gemm_avg * 1e-3) / 1e12
-        bpe = prep_bytes_per_elem(args.fmt, args.mask, has_res)
-        prep_gbs = M * K * bpe / (prep_avg * 1e-3) / 1e9
-        # the committed capture is of the method's kernel (NVFP4, pair 4:8, residual on)
-        method = ((args.fmt, args.mask, args.residual) == ("nvfp4", "pair48", "on")
-                  and not args.given_amax and M == WORKLOADS[args.workload][0])
-        traffic = traffic_from_profile(args.workload) if method else None
-        # the preparation is bound by instruction issue, not HBM: its issue-rate roofline
-        # (warp instructions per element from the committed count; peak = 4 issues per SM
-        # per cycle at the median SM clock of the timed region)
-        ipe = prep_issue_from_profile(args.workload) if method else None
-        issue = None
-        if ipe and clocks.get("sm_mhz"):
-            n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
-            peak_i = n_sm * 4 * clocks["sm_mhz"] * 1e6
-            ach_i = ipe * M * K / (prep_avg * 1e-3)
-            issue = {"warp_instructions_per_elem": ipe, "achieved_ginst_s": ach_i / 1e9,
-                     "peak_ginst_s": peak_i / 1e9, "frac": ach_i / peak_i,
-                     "peak_source": f"{n_sm} SMs x 4 issue slots x {clocks['sm_mhz']} MHz"}
-        line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
-            "data": "synthetic",
-            "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": args.fmt,
-                       "mask": args.mask, "residual": args.residual, "out": "bf16",
-                       "l2": (f"weights rotate over {n_w} copies ({n_w * wbytes / 1e6:.0f} MB "
-                              "> 126 MB L2)") if decode else
-                             (f"{n_sets} rotating input sets ({n_sets * (M * K + M * N) * 2 / 1e6:.0f}"
-                              " MB of X and Y > 126 MB L2)"),
-                       "schedule": ("pipelined: step i+1's preparation beside step i's GEMM "
-                                    "(two streams)") if args.pipeline else "serial",
-                       "launch": ("steps replayed from a CUDA graph (decode-sized calls outrun "
-                                  "host launches)") if decode and not args.pipeline else "eager",
-                       "amax": "given (reduced before the timed region)" if args.given_amax
-                               else "reduced in every call",
-                       "gemm_workspace": "split-K" if WS is not None else "none",
-                       "parallelism": f"dp{world}"},
-            "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": peak,
-                         "unit": "TFLOP/s", "frac": gemm_tflops / peak,
-                         "traffic": traffic,
-                         "peak_source": peak_source,
-                         "ceiling_frac": metric_ceiling(args.mask, has_res),
-                         # the tensor pipe's executed work (sparse backbone at twice the
-                         # dense rate): 2MNK / ceiling per launch, against the same peak
-                         "executed_frac": gemm_tflops / peak / metric_ceiling(args.mask, has_res),
-                         # context: against 4x the sustained bf16 figure and the spec sheet
-                         "frac_vs_sustained_peak": gemm_tflops / (bf16_sus * FP4_OVER_BF16),
-                         "frac_vs_nominal_peak": gemm_tflops / NOMINAL_FP4_TFLOPS,
-                         "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg},
-            "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
-                     "frac": prep_gbs / hbm,
-                     "traffic": prep_traffic_from_profile(args.workload) if method else None,
-                     "frac_vs_nominal_hbm": prep_gbs / NOMINAL_HBM_GBS,
-                     "bytes_per_elem": bpe,
-                     "ms_in_step": prep_in_step,
-                     "issue_roofline": issue,
-                     "kernel": " + ".join(prep_kernels(args.fmt, args.mask, args.residual,
-                                                       args.given_amax)),
-                     "note": ("ms: calls back to back over "
-                              + ("input sets larger than L2 (X read from HBM every call)"
-                                 if n_prep * xb >= 2 * L2_BYTES else
-                                 f"{n_prep} input sets (a few rows: X stays in L2)")
-                              + "; ms_in_step: between events around the call inside the "
-                                "step, which adds the first kernel's launch gap; algorithmic "
-                                "bytes count X once")},
-            "gemm_tflops": gemm_tflops,
-            "pct_fp4_peak": 100.0 * gemm_tflops / peak,
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
-                    "d2h_bytes_per_step": M * N * 2},
-            # split-K (decode-sized M) adds a summing kernel
-            "gpu_launches": (len(prep_kernels(args.fmt, args.mask, args.residual,
-                                              args.given_amax)) + 1 +
-                             (1 if WS is not None and decode else 0)) * args.steps,
-            "clocks": clocks,
-        }
-        if decode:  # below the ridge point the GEMM streams its weight: an HBM roofline
-            gbs = wbytes / (gemm_avg * 1e-3) / 1e9
-            line["roofline"] = {
-                "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                "traffic": None, "peak_source": f"{peak_src}: copy bandwidth",
-                "note": "FP4 weight payload (codes and both scale views) / linear call time "
-                        "(split-K partials summed by a second kernel when the workspace is used)",
-                "weight_bytes": wbytes, "split_k": WS is not None,
-                "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg}
+    hbm, bf16, bf16_sus, peak_src = load_peaks()
+    clocks = clk.summary()
+    peak, peak_source = fp4_peak(clocks.get("sm_mhz"), clocks.get("sm_max_mhz"))
+    gemm_avg = float(np.mean(gemm_ms))
+    prep_avg = prep_b2b
+    prep_in_step = float(np.mean(prep_ms))
+    gemm_tflops = flops / (gemm_avg * 1e-3) / 1e12
+    bpe = prep_bytes_per_elem(args.fmt, args.mask, has_res)
+    prep_gbs = M * K * bpe / (prep_avg * 1e-3) / 1e9
+    # the committed capture is of the method's kernel (NVFP4, pair 4:8, residual on)
+    method = ((args.fmt, args.mask, args.residual) == ("nvfp4", "pair48", "on")
+              and not args.given_amax and M == WORKLOADS[args.workload][0])
+    traffic = traffic_from_profile(args.workload) if method else None
+    # the preparation is bound by instruction issue, not HBM: its issue-rate roofline
+    # (warp instructions per element from the committed count; peak = 4 issues per SM
+    # per cycle at the median SM clock of the timed region)
+    ipe = prep_issue_from_profile(args.workload) if method else None
+    issue = None
+    if ipe and clocks.get("sm_mhz"):
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        peak_i = n_sm * 4 * clocks["sm_mhz"] * 1e6
+        ach_i = ipe * M * K / (prep_avg * 1e-3)
+        issue = {"warp_instructions_per_elem": ipe, "achieved_ginst_s": ach_i / 1e9,
+                 "peak_ginst_s": peak_i / 1e9, "frac": ach_i / peak_i,
+                 "peak_source": f"{n_sm} SMs x 4 issue slots x {clocks['sm_mhz']} MHz"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "format": args.fmt,
+                   "mask": args.mask, "residual": args.residual, "out": "bf16",
+                   "l2": (f"weights rotate over {n_w} copies ({n_w * wbytes / 1e6:.0f} MB "
+                          "> 126 MB L2)") if decode else
+                         (f"{n_sets} rotating input sets ({n_sets * (M * K + M * N) * 2 / 1e6:.0f}"
+                          " MB of X and Y > 126 MB L2)"),
+                   "schedule": ("pipelined: step i+1's preparation beside step i's GEMM "
+                                "(two streams)") if args.pipeline else "serial",
+                   "launch": ("steps replayed from a CUDA graph (decode-sized calls outrun "
+                              "host launches)") if decode and not args.pipeline else "eager",
+                   "amax": "given (reduced before the timed region)" if args.given_amax
+                           else "reduced in every call",
+                   "gemm_workspace": "split-K" if WS is not None else "none",
+                   "parallelism": f"dp{world}"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": gemm_tflops / peak,
+                     "traffic": traffic,
+                     "peak_source": peak_source,
+                     "ceiling_frac": metric_ceiling(args.mask, has_res),
+                     # the tensor pipe's executed work (sparse backbone at twice the
+                     # dense rate): 2MNK / ceiling per launch, against the same peak
+                     "executed_frac": gemm_tflops / peak / metric_ceiling(args.mask, has_res),
+                     # context: against 4x the sustained bf16 figure and the spec sheet
+                     "frac_vs_sustained_peak": gemm_tflops / (bf16_sus * FP4_OVER_BF16),
+                     "frac_vs_nominal_peak": gemm_tflops / NOMINAL_FP4_TFLOPS,
+                     "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg},
+        "prep": {"ms": prep_avg, "gbs": prep_gbs, "hbm_peak_gbs": hbm,
+                 "frac": prep_gbs / hbm,
+                 "traffic": prep_traffic_from_profile(args.workload) if method else None,
+                 "frac_vs_nominal_hbm": prep_gbs / NOMINAL_HBM_GBS,
+                 "bytes_per_elem": bpe,
+                 "ms_in_step": prep_in_step,
+                 "issue_roofline": issue,
+                 "kernel": " + ".join(prep_kernels(args.fmt, args.mask, args.residual,
+                                                   args.given_amax)),
+                 "note": ("ms: calls back to back over "
+                          + ("input sets larger than L2 (X read from HBM every call)"
+                             if n_prep * xb >= 2 * L2_BYTES else
+                             f"{n_prep} input sets (a few rows: X stays in L2)")
+                          + "; ms_in_step: between events around the call inside the "
+                            "step, which adds the first kernel's launch gap; algorithmic "
+                            "bytes count X once")},
+        "gemm_tflops": gemm_tflops,
+        "pct_fp4_peak": 100.0 * gemm_tflops / peak,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * K * 2,
+                "d2h_bytes_per_step": M * N * 2},
+        # split-K (decode-sized M) adds a summing kernel
+        "gpu_launches": (len(prep_kernels(args.fmt, args.mask, args.residual,
+                                          args.given_amax)) + 1 +
+                         (1 if WS is not None and decode else 0)) * args.steps,
+        "clocks": clocks,
+    }
+    if decode:  # below the ridge point the GEMM streams its weight: an HBM roofline
+        gbs = wbytes / (gemm_avg * 1e-3) / 1e9
+        line["roofline"] = {
+            "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+            "traffic": None, "peak_source": f"{peak_src}: copy bandwidth",
+            "note": "FP4 weight payload (codes and both scale views) / linear call time "
+                    "(split-K partials summed by a second kernel when the workspace is used)",
+            "weight_bytes": wbytes, "split_k": WS is not None,
+            "kernel": gemm_kernel_name(M, N, args.residual), "kernel_ms": gemm_avg}
     return line
 
 
