@@ -1,8 +1,15 @@
 """Host-side helpers of bench.py on CPU: the --m override of a workload's token rows, the
-inputs drawn for it, and the oracle's CPU baseline counting only the rows it really ran."""
+inputs drawn for it, the oracle's CPU baseline counting only the rows it really ran, the
+roofline's algorithmic bytes and ceilings, the clock-aware peak, and the gating of the
+committed ncu records by the source they were taken on."""
 import argparse
+import json
+import os
 
+import numpy as np
 import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 @pytest.fixture
@@ -110,3 +117,59 @@ def test_fp4_peak_follows_the_clock_of_the_timed_region(monkeypatch):
     assert p == pytest.approx(4 * 1654.2)
     monkeypatch.setattr(bench, "sustained_clock_mhz", lambda: None)
     assert bench.fp4_peak(1515.0, 1965.0)[0] == pytest.approx(4 * 1654.2)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("mask", ["pair48", "elem24", "none"])
+@pytest.mark.parametrize("residual", [True, False])
+def test_prep_bytes_per_elem_is_the_output_layout(fmt, mask, residual):
+    """The preparation roofline's algorithmic bytes per element = the 16-bit read plus every
+    byte of the oracle's output buffers (a shape without tile padding: 128 rows, K / block a
+    multiple of 4)."""
+    import bench
+    from oracle import sharq as S
+    M, K = 128, 512
+    x = np.random.default_rng(1).standard_normal((M, K)).astype(np.float32)
+    bufs = S.act_buffers(S.prepare(x, fmt, mask, residual=residual))
+    out = sum(v.size for k, v in bufs.items() if k != "tensor_scale" and v is not None)
+    assert bench.prep_bytes_per_elem(fmt, mask, residual) == pytest.approx(2.0 + out / (M * K))
+
+
+def test_metric_ceiling_from_the_mma_rates():
+    """2MNK / t at full tensor-pipe use over the dense FP4 peak: the sparse backbone runs at
+    twice the dense rate, a dense residual adds its own pass."""
+    import bench
+    assert bench.metric_ceiling("pair48", True) == pytest.approx(2 / 3)
+    assert bench.metric_ceiling("pair48", False) == pytest.approx(2.0)
+    assert bench.metric_ceiling("elem24", True) == pytest.approx(0.5)
+    assert bench.metric_ceiling("none", False) == pytest.approx(1.0)
+
+
+def test_gemm_kernel_choice():
+    import bench
+    assert bench.gemm_kernel_name(256, 4096) == "sharq_gemm_pair_kernel"
+    assert bench.gemm_kernel_name(8192, 28672) == "sharq_gemm_pair_kernel"
+    assert bench.gemm_kernel_name(255, 4096) == "sharq_gemm_kernel"     # decode-sized rows
+    assert bench.gemm_kernel_name(4096, 384) == "sharq_gemm_kernel"     # N not a multiple of 256
+    assert bench.gemm_kernel_name(4096, 4096, "own") == "sharq_gemm_kernel"  # two accumulators
+
+
+def test_traffic_records_follow_the_code_not_the_comments(tmp_path, monkeypatch):
+    """A committed ncu record is reported only while it matches the hash of the GEMM sources;
+    comment and spacing edits keep the hash, a code edit drops the record."""
+    import shutil
+    import bench
+    for f in bench.GEMM_SRC:
+        (tmp_path / f).parent.mkdir(parents=True, exist_ok=True)
+        shutil.copy(os.path.join(ROOT, f), tmp_path / f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    rec = {"mlp_gate_up": {"dram_bytes_per_launch": 123, "gemm_src": bench.src_hash(bench.GEMM_SRC)}}
+    (tmp_path / "profiles" / "gemm_traffic.json").write_text(json.dumps(rec))
+    assert bench.traffic_from_profile("mlp_gate_up") == 123
+    assert bench.traffic_from_profile("attn_proj") is None           # no record for it
+    src = tmp_path / bench.GEMM_SRC[0]
+    src.write_text(src.read_text() + "\n// a note\n/* and another */\n\n")
+    assert bench.traffic_from_profile("mlp_gate_up") == 123           # comments only
+    src.write_text(src.read_text() + "\nstatic int sharq_extra_symbol = 1;\n")
+    assert bench.traffic_from_profile("mlp_gate_up") is None          # the code changed
